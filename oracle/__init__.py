@@ -1,0 +1,144 @@
+"""CPU oracle for the FP8 block-scaled NT GEMM (dense / contiguous / masked).
+
+TEST INFRASTRUCTURE ONLY: imported by ``tests/``, ``__graft_entry__.smoke()``
+and the CPU-baseline leg of ``bench.py``; never by the library.  It shares no
+code with the CUDA path.  The arithmetic lives in ``oracle.c`` (plain C, FP64,
+OpenMP over output rows); this module compiles it with gcc and marshals numpy
+arrays.  ``brute.py`` is a second, pure-Python statement of the same
+definition for tiny shapes.
+
+Definition (DeepGEMM pages, page 2 "技术特性" and page 3 "核心功能"):
+    D[m,n] = sum_kb sA[m,kb] * sB[n//128,kb] * sum_{k in kb} A[m,k] * B[n,k]
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from typing import Optional
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "oracle.c")
+_LIB_PATH = os.path.join(_HERE, "_oracle.so")
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile oracle.c into _oracle.so (gcc, -O3, OpenMP, portable x86-64)."""
+    if (not force and os.path.exists(_LIB_PATH)
+            and os.path.getmtime(_LIB_PATH) >= os.path.getmtime(_SRC)):
+        return _LIB_PATH
+    tmp = _LIB_PATH + f".tmp{os.getpid()}"
+    subprocess.check_call(["gcc", "-O3", "-fopenmp", "-fPIC", "-shared", "-std=c11",
+                           "-o", tmp, _SRC, "-lm"])
+    os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        # ORACLE_SO lets the mutation test point the wrapper at a deliberately
+        # broken build of oracle.c; it is never set otherwise.
+        lib = ctypes.CDLL(os.environ.get("ORACLE_SO") or build())
+        P = ctypes.c_void_p
+        L = ctypes.c_long
+        lib.oracle_e4m3_table.argtypes = [P]
+        lib.oracle_e4m3_table.restype = None
+        lib.oracle_fp8_gemm_nt.argtypes = [P, P, L, P, P, L, L, L, P]
+        lib.oracle_m_grouped_contiguous.argtypes = [P, P, L, P, P, P, L, L, L, L, P]
+        lib.oracle_m_grouped_masked.argtypes = [P, P, L, P, P, P, L, L, L, L, P]
+        lib.oracle_points.argtypes = [ctypes.c_int, P, P, L, P, P, P, P, L, L, L, L,
+                                      L, P, P, P, P]
+        for f in ("oracle_fp8_gemm_nt", "oracle_m_grouped_contiguous",
+                  "oracle_m_grouped_masked", "oracle_points"):
+            getattr(lib, f).restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+def _p(x: Optional[np.ndarray]):
+    return None if x is None else x.ctypes.data_as(ctypes.c_void_p)
+
+
+def _c(x, dtype):
+    return np.ascontiguousarray(x, dtype=dtype)
+
+
+def e4m3_table() -> np.ndarray:
+    """The oracle's 256-entry E4M3 decode table (float64)."""
+    out = np.empty(256, dtype=np.float64)
+    _load().oracle_e4m3_table(_p(out))
+    return out
+
+
+def gemm_dense(a, sfa, ld_sfa, b, sfb, M, N, K) -> np.ndarray:
+    """Dense D = A * B^T with block scales; returns float64 [M, N]."""
+    a, b = _c(a, np.uint8), _c(b, np.uint8)
+    sfa, sfb = _c(sfa, np.float32), _c(sfb, np.float32)
+    d = np.empty((M, N), dtype=np.float64)
+    rc = _load().oracle_fp8_gemm_nt(_p(a), _p(sfa), ld_sfa, _p(b), _p(sfb), M, N, K, _p(d))
+    if rc:
+        raise ValueError(f"oracle_fp8_gemm_nt rejected the shape (rc={rc})")
+    return d
+
+
+def gemm_contiguous(a, sfa, ld_sfa, b, sfb, m_indices, M_total, N, K, G,
+                    fill: float = np.nan) -> np.ndarray:
+    """M-grouped contiguous; padding rows (m_indices < 0) hold ``fill``."""
+    a, b = _c(a, np.uint8), _c(b, np.uint8)
+    sfa, sfb = _c(sfa, np.float32), _c(sfb, np.float32)
+    mi = _c(m_indices, np.int32)
+    d = np.full((M_total, N), fill, dtype=np.float64)
+    rc = _load().oracle_m_grouped_contiguous(_p(a), _p(sfa), ld_sfa, _p(b), _p(sfb),
+                                             _p(mi), M_total, N, K, G, _p(d))
+    if rc:
+        raise ValueError(f"oracle_m_grouped_contiguous rejected the input (rc={rc})")
+    return d
+
+
+def gemm_masked(a, sfa, ld_sfa, b, sfb, masked_m, G, Mmax, N, K,
+                fill: float = np.nan) -> np.ndarray:
+    """M-grouped masked; rows >= masked_m[g] hold ``fill``.  Returns [G, Mmax, N]."""
+    a, b = _c(a, np.uint8), _c(b, np.uint8)
+    sfa, sfb = _c(sfa, np.float32), _c(sfb, np.float32)
+    mm = _c(masked_m, np.int32)
+    d = np.full((G, Mmax, N), fill, dtype=np.float64)
+    rc = _load().oracle_m_grouped_masked(_p(a), _p(sfa), ld_sfa, _p(b), _p(sfb), _p(mm),
+                                         G, Mmax, N, K, _p(d))
+    if rc:
+        raise ValueError(f"oracle_m_grouped_masked rejected the input (rc={rc})")
+    return d
+
+
+_LAYOUT_CODE = {"dense": 0, "contiguous": 1, "masked": 2}
+
+
+def points(prob, grp, row, col) -> np.ndarray:
+    """Sampled outputs D[grp, row, col] of a ``workloads.Problem``."""
+    a, b = _c(prob.a, np.uint8), _c(prob.b, np.uint8)
+    sfa, sfb = _c(prob.sfa, np.float32), _c(prob.sfb, np.float32)
+    mi = None if prob.m_indices is None else _c(prob.m_indices, np.int32)
+    mm = None if prob.masked_m is None else _c(prob.masked_m, np.int32)
+    grp, row, col = (_c(x, np.int32) for x in (grp, row, col))
+    out = np.empty(len(row), dtype=np.float64)
+    rc = _load().oracle_points(_LAYOUT_CODE[prob.layout], _p(a), _p(sfa), prob.ld_sfa,
+                               _p(b), _p(sfb), _p(mi), _p(mm), prob.G, prob.M, prob.N,
+                               prob.K, len(row), _p(grp), _p(row), _p(col), _p(out))
+    if rc:
+        raise ValueError(f"oracle_points rejected the input (rc={rc})")
+    return out
+
+
+def solve(prob) -> np.ndarray:
+    """Full oracle output for a ``workloads.Problem`` (float64, NaN where unwritten)."""
+    if prob.layout == "dense":
+        return gemm_dense(prob.a, prob.sfa, prob.ld_sfa, prob.b[0], prob.sfb[0],
+                          prob.M, prob.N, prob.K)
+    if prob.layout == "contiguous":
+        return gemm_contiguous(prob.a, prob.sfa, prob.ld_sfa, prob.b, prob.sfb,
+                               prob.m_indices, prob.M, prob.N, prob.K, prob.G)
+    return gemm_masked(prob.a, prob.sfa, prob.ld_sfa, prob.b, prob.sfb, prob.masked_m,
+                       prob.G, prob.M, prob.N, prob.K)

@@ -1,0 +1,47 @@
+"""The oracle's pins must catch plausible mistakes.
+
+Each case plants one mistake in a temporary copy of oracle/oracle.c (on the
+CPU; the repository's oracle is untouched), builds it, and runs the pin suite
+against it in a subprocess: the suite must FAIL for every mutant.
+"""
+import os
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+MUTANTS = {
+    "weight block index n%128 instead of n/128":
+        ("n / ORC_BLOCK) * KB, K, lut);", "n % ORC_BLOCK) * KB, K, lut);"),
+    "last K-block dropped":
+        ("for (long kb = 0; kb < KB; ++kb) {", "for (long kb = 0; kb + 1 < KB; ++kb) {"),
+    "activation scales read row-major":
+        ("sa[kb * sa_stride]", "sa[kb]"),
+    "subnormal exponent off by one":
+        ("v = ldexp((double)mantissa / 8.0, 1 - 7);", "v = ldexp((double)mantissa / 8.0, 0 - 7);"),
+    "sign bit ignored":
+        ("lut[code] = sign ? -v : v;", "lut[code] = v;"),
+    "K index of B shifted":
+        ("p += lut[ak[i]] * lut[bk[i]];", "p += lut[ak[i]] * lut[bk[(i + 1) % ORC_BLOCK]];"),
+    "weight scale ignored":
+        ("((double)sa[kb * sa_stride] * (double)sb[kb]) * p", "((double)sa[kb * sa_stride]) * p"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_catch_mutant(name, tmp_path):
+    old, new = MUTANTS[name]
+    src = open(os.path.join(ROOT, "oracle", "oracle.c")).read()
+    assert src.count(old) >= 1, "mutation site not found"
+    mutated = tmp_path / "oracle_mutant.c"
+    mutated.write_text(src.replace(old, new))
+    so = tmp_path / "oracle_mutant.so"
+    subprocess.check_call(["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11",
+                           "-o", str(so), str(mutated), "-lm"])
+    env = dict(os.environ, ORACLE_SO=str(so))
+    r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
+                        os.path.join(ROOT, "tests", "test_oracle.py")],
+                       cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
+    assert r.returncode != 0, f"pins did not catch: {name}\n{r.stdout[-2000:]}"

@@ -1,0 +1,279 @@
+"""Seeded synthetic inputs for the FP8 block-scaled NT GEMM.
+
+This module is shared by the oracle side and the CUDA side of the tests and by
+``bench.py``.  It draws random numbers and packs them into the storage formats
+the library consumes; it holds none of the GEMM's arithmetic (no E4M3 decode,
+no dot products, no promotion).  The FP8 encoding of a float uses torch's own
+``float8_e4m3fn`` cast (round-to-nearest-even, OCP E4M3 "fn" format), a library
+primitive.
+
+Storage formats (shared with the C ABI):
+
+* ``a``   uint8 E4M3 bytes, [rows, K] row-major (K-major).
+* ``sfa`` float32 [KB, ld_sfa] "MN-major": for K-block kb, one float per row;
+  ``ld_sfa`` = rows rounded up to a multiple of 4 (16-byte TMA alignment).
+  Masked layout: [G, KB, ld_sfa].
+* ``b``   uint8 E4M3 bytes, [G, N, K] row-major (G = 1 for dense).
+* ``sfb`` float32 [G, NB, KB] row-major, one float per 128x128 block.
+
+Quantisation recipe (the pages only say "fine-grained" / "block-wise" scaling,
+DeepGEMM pages 2 and 3 "技术特性" / "精细粒度缩放"; the 1x128 and 128x128 block
+shapes come from the workload definitions): per block, s = amax / 448 in FP32
+(s = 1 when the block is all zero), q = e4m3_rne(clamp(x / s, -448, 448)).
+
+Random streams use ``numpy.random.default_rng`` (PCG64).  Dense: A, then B,
+then the outlier columns, all from ``seed``.  Grouped layouts: the structure
+(multinomial token counts, masked counts) comes from ``seed`` because it fixes
+the operand shapes; A and then B come from ``seed + 1000``.
+"""
+from __future__ import annotations
+
+import dataclasses
+from typing import Optional
+
+import numpy as np
+import torch
+
+BLOCK = 128            # K-block and weight-block edge
+E4M3_MAX = 448.0
+NAN_BYTE = 0x7F        # an E4M3 NaN code, used to poison padding rows
+ALIGN_M = 128          # row alignment of the contiguous layout
+
+
+def tma_aligned(n: int, elem_bytes: int = 4) -> int:
+    """Round n up so that n * elem_bytes is a multiple of 16 bytes."""
+    q = 16 // elem_bytes
+    return (n + q - 1) // q * q
+
+
+def _to_e4m3_bytes(x: torch.Tensor) -> torch.Tensor:
+    x = torch.clamp(x, -E4M3_MAX, E4M3_MAX)
+    return x.to(torch.float8_e4m3fn).view(torch.uint8)
+
+
+def quantize_rows_1x128(x: np.ndarray):
+    """Per-row, per-128-K block quantisation.  x: float32 [R, K].
+
+    Returns (q uint8 [R, K], s float32 [R, KB])."""
+    R, K = x.shape
+    assert K % BLOCK == 0
+    t = torch.from_numpy(x).view(R, K // BLOCK, BLOCK)
+    amax = t.abs().amax(dim=2)
+    s = amax / E4M3_MAX
+    s = torch.where(amax == 0, torch.ones_like(s), s)
+    q = _to_e4m3_bytes(t / s.unsqueeze(2)).reshape(R, K)
+    return q.numpy(), s.numpy().astype(np.float32)
+
+
+def quantize_blocks_128x128(x: np.ndarray):
+    """Per-128x128 block quantisation.  x: float32 [N, K] (N may have a tail).
+
+    Returns (q uint8 [N, K], s float32 [NB, KB])."""
+    N, K = x.shape
+    assert K % BLOCK == 0
+    NB, KB = (N + BLOCK - 1) // BLOCK, K // BLOCK
+    t = torch.from_numpy(x)
+    pad = NB * BLOCK - N
+    tp = torch.nn.functional.pad(t, (0, 0, 0, pad)) if pad else t
+    blk = tp.view(NB, BLOCK, KB, BLOCK)
+    amax = blk.abs().amax(dim=(1, 3))                  # [NB, KB]
+    s = amax / E4M3_MAX
+    s = torch.where(amax == 0, torch.ones_like(s), s)
+    q = _to_e4m3_bytes(blk / s[:, None, :, None]).reshape(NB * BLOCK, K)[:N]
+    return q.contiguous().numpy(), s.numpy().astype(np.float32)
+
+
+def sfa_mn_major(s_rows: np.ndarray, ld: Optional[int] = None) -> np.ndarray:
+    """[R, KB] per-row scales -> [KB, ld] MN-major storage (padding = 0)."""
+    R, KB = s_rows.shape
+    ld = tma_aligned(R) if ld is None else ld
+    out = np.zeros((KB, ld), dtype=np.float32)
+    out[:, :R] = s_rows.T
+    return out
+
+
+@dataclasses.dataclass
+class Problem:
+    """One GEMM problem in the library's storage formats (host numpy arrays)."""
+    layout: str                    # "dense" | "contiguous" | "masked"
+    M: int                         # dense: rows; contiguous: M_total; masked: Mmax
+    N: int
+    K: int
+    G: int
+    a: np.ndarray                  # uint8
+    sfa: np.ndarray                # float32
+    ld_sfa: int
+    b: np.ndarray                  # uint8 [G, N, K]
+    sfb: np.ndarray                # float32 [G, NB, KB]
+    m_indices: Optional[np.ndarray] = None   # int32 [M_total] (contiguous)
+    masked_m: Optional[np.ndarray] = None    # int32 [G] (masked)
+    name: str = ""
+
+    @property
+    def KB(self) -> int:
+        return self.K // BLOCK
+
+    @property
+    def NB(self) -> int:
+        return (self.N + BLOCK - 1) // BLOCK
+
+    def valid_rows(self) -> int:
+        if self.layout == "dense":
+            return self.M
+        if self.layout == "contiguous":
+            return int((self.m_indices >= 0).sum())
+        return int(self.masked_m.sum())
+
+    def groups_touched(self) -> int:
+        if self.layout == "dense":
+            return 1
+        if self.layout == "contiguous":
+            return int(len(np.unique(self.m_indices[self.m_indices >= 0])))
+        return int((self.masked_m > 0).sum())
+
+    def flops(self) -> float:
+        """Algorithmic FLOP: 2 * valid rows * N * K."""
+        return 2.0 * self.valid_rows() * self.N * self.K
+
+    def bytes(self) -> float:
+        """Algorithmic bytes: A + B + sA + sB + D over valid rows / touched groups."""
+        rows, g = self.valid_rows(), self.groups_touched()
+        return float(rows * self.K + g * self.N * self.K + rows * self.KB * 4
+                     + g * self.NB * self.KB * 4 + rows * self.N * 2)
+
+    def d_shape(self):
+        if self.layout == "masked":
+            return (self.G, self.M, self.N)
+        return (self.M, self.N)
+
+
+def _normal(rng, shape):
+    return rng.standard_normal(shape, dtype=np.float32)
+
+
+def make_dense(M: int, N: int, K: int, seed: int, outliers: bool = False,
+               name: str = "") -> Problem:
+    """Dense problem: A ~ N(0,1) [M,K], B ~ N(0,1) [N,K].
+
+    With ``outliers``, one fixed set of floor(0.01*K) K-columns of A (drawn
+    after A and B) is multiplied by 20 before quantisation."""
+    rng = np.random.default_rng(seed)
+    a32 = _normal(rng, (M, K))
+    b32 = _normal(rng, (N, K))
+    if outliers:
+        cols = rng.choice(K, size=K // 100, replace=False)
+        a32[:, cols] *= 20.0
+    qa, sa = quantize_rows_1x128(a32) if M > 0 else (np.zeros((0, K), np.uint8),
+                                                     np.zeros((0, K // BLOCK), np.float32))
+    qb, sb = quantize_blocks_128x128(b32)
+    ld = tma_aligned(max(M, 1))
+    return Problem("dense", M, N, K, 1, qa, sfa_mn_major(sa, ld), ld,
+                   qb[None], sb[None], name=name)
+
+
+def make_contiguous(counts, N: int, K: int, seed: int, name: str = "",
+                    poison: bool = True) -> Problem:
+    """M-grouped contiguous problem with explicit per-group token counts.
+
+    Group g's rows are packed back to back and padded to a multiple of 128;
+    padding rows carry m_indices = -1, NaN bytes in A and NaN scales."""
+    rng = np.random.default_rng(seed)
+    counts = [int(c) for c in counts]
+    G = len(counts)
+    padded = [(c + ALIGN_M - 1) // ALIGN_M * ALIGN_M for c in counts]
+    M_total = int(sum(padded))
+    a32 = _normal(rng, (sum(counts), K))
+    b32 = _normal(rng, (G * N, K))
+    m_idx = np.full((M_total,), -1, dtype=np.int32)
+    qa_all, sa_all = (quantize_rows_1x128(a32) if a32.shape[0] else
+                      (np.zeros((0, K), np.uint8), np.zeros((0, K // BLOCK), np.float32)))
+    a = np.full((M_total, K), NAN_BYTE if poison else 0, dtype=np.uint8)
+    sa = np.full((M_total, K // BLOCK), np.nan if poison else 0.0, dtype=np.float32)
+    src = dst = 0
+    for g, (c, p) in enumerate(zip(counts, padded)):
+        a[dst:dst + c] = qa_all[src:src + c]
+        sa[dst:dst + c] = sa_all[src:src + c]
+        m_idx[dst:dst + c] = g
+        src += c
+        dst += p
+    qb = np.empty((G, N, K), dtype=np.uint8)
+    NB = (N + BLOCK - 1) // BLOCK
+    sb = np.empty((G, NB, K // BLOCK), dtype=np.float32)
+    for g in range(G):
+        qb[g], sb[g] = quantize_blocks_128x128(b32[g * N:(g + 1) * N])
+    ld = tma_aligned(max(M_total, 1))
+    sfa = sfa_mn_major(sa, ld)
+    if poison:
+        sfa[:, M_total:] = np.nan
+    return Problem("contiguous", M_total, N, K, G, a, sfa, ld, qb, sb,
+                   m_indices=m_idx, name=name)
+
+
+def make_contiguous_multinomial(G: int, tokens: int, N: int, K: int, seed: int,
+                                name: str = "") -> Problem:
+    """Token counts per expert from multinomial(tokens, [1/G]*G) drawn from a
+    generator seeded with ``seed`` before the operands (structure first here
+    because the counts fix the operand shapes); operands then come from
+    ``seed + 1000``."""
+    rng = np.random.default_rng(seed)
+    counts = rng.multinomial(tokens, [1.0 / G] * G)
+    return make_contiguous(counts, N, K, seed + 1000, name=name)
+
+
+def make_masked(masked_m, Mmax: int, N: int, K: int, seed: int, name: str = "",
+                poison: bool = True) -> Problem:
+    """M-grouped masked problem: A [G, Mmax, K], valid rows m < masked_m[g].
+
+    Rows >= masked_m[g] carry NaN bytes and NaN scales."""
+    rng = np.random.default_rng(seed)
+    masked_m = np.asarray(masked_m, dtype=np.int32)
+    G = len(masked_m)
+    a32 = _normal(rng, (G * Mmax, K))
+    b32 = _normal(rng, (G * N, K))
+    qa, sa = quantize_rows_1x128(a32)
+    qa = qa.reshape(G, Mmax, K)
+    sa = sa.reshape(G, Mmax, K // BLOCK)
+    ld = tma_aligned(Mmax)
+    sfa = np.zeros((G, K // BLOCK, ld), dtype=np.float32)
+    for g in range(G):
+        sfa[g, :, :Mmax] = sa[g].T
+        if poison:
+            qa[g, masked_m[g]:] = NAN_BYTE
+            sfa[g, :, masked_m[g]:] = np.nan
+    qb = np.empty((G, N, K), dtype=np.uint8)
+    NB = (N + BLOCK - 1) // BLOCK
+    sb = np.empty((G, NB, K // BLOCK), dtype=np.float32)
+    for g in range(G):
+        qb[g], sb[g] = quantize_blocks_128x128(b32[g * N:(g + 1) * N])
+    return Problem("masked", Mmax, N, K, G, qa, sfa, ld, qb, sb,
+                   masked_m=masked_m, name=name)
+
+
+def make_masked_uniform(G: int, Mmax: int, N: int, K: int, seed: int,
+                        name: str = "") -> Problem:
+    """masked_m[g] ~ Uniform{0..Mmax} from ``seed``; operands from seed+1000."""
+    rng = np.random.default_rng(seed)
+    masked_m = rng.integers(0, Mmax + 1, size=G).astype(np.int32)
+    return make_masked(masked_m, Mmax, N, K, seed + 1000, name=name)
+
+
+# The five workloads of the method's benchmark set (shapes from the pages'
+# benchmark table, DeepGEMM page 2 "性能实测", plus the expert counts).
+WORKLOADS = {
+    "dense_tiny": dict(kind="dense", M=128, N=256, K=512, seed=0),
+    "dense_decode_m64": dict(kind="dense", M=64, N=2112, K=7168, seed=1, outliers=True),
+    "dense_decode_m128": dict(kind="dense", M=128, N=2112, K=7168, seed=2, outliers=True),
+    "dense_large": dict(kind="dense", M=4096, N=7168, K=16384, seed=3),
+    "contiguous_g4": dict(kind="contiguous", G=4, tokens=32768, N=4096, K=7168, seed=4),
+    "masked_g16": dict(kind="masked", G=16, Mmax=256, N=4096, K=7168, seed=5),
+}
+
+
+def make_workload(name: str) -> Problem:
+    w = dict(WORKLOADS[name])
+    kind = w.pop("kind")
+    if kind == "dense":
+        return make_dense(name=name, **w)
+    if kind == "contiguous":
+        return make_contiguous_multinomial(w["G"], w["tokens"], w["N"], w["K"], w["seed"], name=name)
+    return make_masked_uniform(w["G"], w["Mmax"], w["N"], w["K"], w["seed"], name=name)
