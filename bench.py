@@ -1,0 +1,404 @@
+"""Benchmark of the FP8 block-scaled NT GEMM on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step = one call of the hot path (scheduling, TMA loads, tcgen05 MMA,
+per-K-block promotion, epilogue; swap-AB and split-K for small M) on one
+batch of seeded synthetic inputs already resident in HBM.  L2 is flushed
+(a 512 MB write) before every timed step and the step is timed alone with CUDA
+events on the launching stream.  Multi-GPU (torchrun): each rank runs its own
+independent problem (no collective on the data path, weak scaling); the step
+time is the max over ranks.  ``--impl reference`` times the CPU oracle (FP64,
+all host cores) on a bounded sample of the same workload instead.
+
+Prints ONE JSON line on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "FP8 TFLOPS and HBM GB/s per shape, % of B200 FP8/HBM roofline, 1 GPU"
+DEFAULT_WORKLOAD = "dense_decode_m64"
+# The pages' own figure for the exact same workload (H800, another machine:
+# context only).  DeepGEMM page 2 "性能实测": M=64 N=2112 K=7168 -> 1688 GB/s.
+PAGES_NUMBER = {"dense_decode_m64": (1688.0, "GB/s")}
+UNIT = {"dense_tiny": "TFLOP/s", "dense_decode_m64": "GB/s", "dense_decode_m128": "GB/s",
+        "dense_large": "TFLOP/s", "contiguous_g4": "TFLOP/s", "masked_g16": "GB/s"}
+KERNEL_SOURCES = ["moe_grouped_gemm_fp32_b200/csrc/gemm_kernel.cuh",
+                  "moe_grouped_gemm_fp32_b200/csrc/ptx.cuh",
+                  "moe_grouped_gemm_fp32_b200/csrc/dg_api.cu"]
+FLUSH_BYTES = 512 << 20
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as fh:
+            return json.load(fh), "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+def profiled_traffic(workload: str):
+    """DRAM bytes per launch from the committed ncu summary of this workload,
+    or None when there is none or the kernel sources changed since."""
+    p = os.path.join(ROOT, "profiles", f"fp8_gemm_kernel_{workload}.md")
+    if not os.path.exists(p):
+        return None
+    text = open(p).read()
+    m = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
+    h = re.search(r"kernel_source_hash:\s*([0-9a-f]+)", text)
+    if not m or not h or h.group(1) != kernel_source_hash():
+        return None
+    return float(m.group(1))
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons, sampled in the background."""
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: str):
+        self.gpu = gpu_index
+        self.samples = []
+        self.proc = None
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) == 7:
+                self.samples.append(parts)
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+        if self.thread is not None:
+            self.thread.join(timeout=5)
+        if not self.samples:
+            return None
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        sm = [num(s[0]) for s in self.samples if num(s[0]) is not None]
+        mx = [num(s[1]) for s in self.samples if num(s[1]) is not None]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for s in self.samples for i in range(4)
+                          if s[3 + i].lower() in ("active", "1")})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(self.samples)}
+
+
+# ----------------------------------------------------------------------------- our arm
+def run_ours(args, rank, world, local_rank):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+    import workloads as W
+    import moe_grouped_gemm_fp32_b200 as dg
+    from moe_grouped_gemm_fp32_b200 import build as dg_build
+
+    dg_build.build()
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    prob = W.make_workload(args.workload)
+    if rank:
+        # independent problem per rank (same shapes, different values)
+        spec = dict(W.WORKLOADS[args.workload])
+        spec["seed"] = spec["seed"] + 7919 * rank
+        kind = spec.pop("kind")
+        if kind == "dense":
+            prob = W.make_dense(**spec)
+        elif kind == "contiguous":
+            prob = W.make_contiguous_multinomial(spec["G"], spec["tokens"], spec["N"], spec["K"], spec["seed"])
+        else:
+            prob = W.make_masked_uniform(spec["G"], spec["Mmax"], spec["N"], spec["K"], spec["seed"])
+
+    host = {k: torch.from_numpy(np.ascontiguousarray(v)).pin_memory()
+            for k, v in (("a", prob.a), ("sfa", prob.sfa), ("b", prob.b), ("sfb", prob.sfb))}
+    if prob.m_indices is not None:
+        host["m_indices"] = torch.from_numpy(prob.m_indices).pin_memory()
+    if prob.masked_m is not None:
+        host["masked_m"] = torch.from_numpy(prob.masked_m).pin_memory()
+    devt = {k: v.to(dev, non_blocking=False) for k, v in host.items()}
+    d = torch.empty(prob.d_shape(), dtype=torch.bfloat16, device=dev)
+    d_host = torch.empty(prob.d_shape(), dtype=torch.bfloat16).pin_memory()
+    flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def call(t, out):
+        if prob.layout == "dense":
+            dg.dg_fp8_gemm_nt(t["a"], t["sfa"], t["b"][0], t["sfb"][0], out, stream)
+        elif prob.layout == "contiguous":
+            dg.dg_m_grouped_fp8_gemm_nt_contiguous(t["a"], t["sfa"], t["b"], t["sfb"], out,
+                                                   t["m_indices"], stream)
+        else:
+            dg.dg_m_grouped_fp8_gemm_nt_masked(t["a"], t["sfa"], t["b"], t["sfb"], out,
+                                               t["masked_m"], stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier(device_ids=[local_rank])
+        torch.cuda.synchronize(dev)
+
+    visible = [v.strip() for v in os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",") if v.strip()]
+    sampler = ClockSampler(visible[local_rank] if local_rank < len(visible) else str(local_rank))
+    # ---- device-resident timing
+    for _ in range(args.warmup):
+        flush.fill_(1.0)
+        call(devt, d)
+    dg.dg_get_device_status(clear=True)
+    sampler.start()
+    barrier()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    for i in range(args.steps):
+        flush.fill_(float(i))            # > L2: every step starts from HBM
+        starts[i].record(stream)
+        call(devt, d)
+        ends[i].record(stream)
+    barrier()
+    clocks = sampler.stop()
+    per_step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    ms = sum(per_step_ms) / len(per_step_ms)
+    status = dg.dg_get_device_status(clear=True)
+    if status:
+        raise RuntimeError(f"kernel status word {status:#x}")
+
+    # ---- end to end through the public API from pinned host buffers
+    for _ in range(max(1, args.warmup // 2)):
+        tt = {k: v.to(dev, non_blocking=True) for k, v in host.items()}
+        call(tt, d)
+        d_host.copy_(d, non_blocking=True)
+    barrier()
+    e_start = torch.cuda.Event(enable_timing=True)
+    e_end = torch.cuda.Event(enable_timing=True)
+    e2e_steps = max(1, min(args.steps, 50))
+    e_start.record(stream)
+    for _ in range(e2e_steps):
+        tt = {k: v.to(dev, non_blocking=True) for k, v in host.items()}
+        call(tt, d)
+        d_host.copy_(d, non_blocking=True)
+    e_end.record(stream)
+    barrier()
+    e2e_ms = e_start.elapsed_time(e_end) / e2e_steps
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    d2h = d.numel() * d.element_size()
+
+    # ---- max over ranks
+    if world > 1:
+        t = torch.tensor([ms, e2e_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms, e2e_ms = t.tolist()
+    return prob, ms, e2e_ms, h2d, d2h, clocks
+
+
+def metric_value(prob, unit, ms, world):
+    if unit == "GB/s":
+        return prob.bytes() * world / (ms * 1e-3) / 1e9
+    return prob.flops() * world / (ms * 1e-3) / 1e12
+
+
+def cpu_baseline(prob, unit, budget_s=10.0):
+    """The oracle as it stands (FP64, OpenMP over all host cores) on a bounded
+    sample: whole problems repeated until ~budget_s, or a leading slice of the
+    output rows when one whole problem would take longer."""
+    import numpy as np
+    import oracle
+    oracle.build()
+    cores = len(os.sched_getaffinity(0))
+    t0 = time.perf_counter()
+    probe_rows = max(1, min(prob.M, 8))
+    if prob.layout == "masked":
+        g = int(np.argmax(prob.masked_m))
+        rows = np.arange(min(probe_rows, int(prob.masked_m[g])))
+        grp = np.full(len(rows) * prob.N, g)
+    else:
+        valid = np.flatnonzero(prob.m_indices >= 0) if prob.layout == "contiguous" else np.arange(prob.M)
+        rows = valid[:probe_rows]
+        grp = np.zeros(len(rows) * prob.N, np.int64)
+    rr = np.repeat(rows, prob.N)
+    cc = np.tile(np.arange(prob.N), len(rows))
+    oracle.points(prob, grp, rr, cc)
+    t_probe = time.perf_counter() - t0
+    per_row = t_probe / len(rows)
+    full_rows = prob.valid_rows()
+    if per_row * full_rows <= budget_s:
+        reps, t0 = 0, time.perf_counter()
+        while True:
+            oracle.solve(prob)
+            reps += 1
+            if time.perf_counter() - t0 >= budget_s:
+                break
+        secs = (time.perf_counter() - t0) / reps
+        sample = f"{reps} full solve(s) of the workload, {secs:.3f} s each"
+    else:
+        n_rows = max(1, int(budget_s / per_row))
+        if prob.layout == "masked":
+            sel = [(g, r) for g in range(prob.G) for r in range(int(prob.masked_m[g]))]
+            sel = sel[:: max(1, len(sel) // n_rows)][:n_rows]
+            grp = np.repeat([s[0] for s in sel], prob.N)
+            rr = np.repeat([s[1] for s in sel], prob.N)
+        else:
+            valid = np.flatnonzero(prob.m_indices >= 0) if prob.layout == "contiguous" else np.arange(prob.M)
+            pick = valid[:: max(1, len(valid) // n_rows)][:n_rows]
+            grp = np.zeros(len(pick) * prob.N, np.int64)
+            rr = np.repeat(pick, prob.N)
+        n_rows = len(rr) // prob.N
+        cc = np.tile(np.arange(prob.N), n_rows)
+        t0 = time.perf_counter()
+        oracle.points(prob, grp, rr, cc)
+        dt = time.perf_counter() - t0
+        secs = dt * full_rows / n_rows
+        sample = (f"{n_rows} of {full_rows} valid output rows (all N columns), "
+                  f"{dt:.1f} s, scaled linearly to the whole workload")
+    value = (prob.bytes() / secs / 1e9) if unit == "GB/s" else (prob.flops() / secs / 1e12)
+    return {"value": value, "unit": unit, "cores": cores, "kind": "oracle", "sample": sample,
+            "seconds_per_step": secs}
+
+
+def run_reference(args, rank, world):
+    import workloads as W
+    if rank != 0:
+        return 0
+    prob = W.make_workload(args.workload)
+    unit = UNIT[args.workload]
+    # per-step CPU budget: the whole --steps/--warmup run stays within a few minutes
+    budget = max(0.2, min(6.0, 150.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        cpu_baseline(prob, unit, budget_s=budget)
+    vals = [cpu_baseline(prob, unit, budget_s=budget) for _ in range(args.steps)]
+    secs = sum(v["seconds_per_step"] for v in vals) / len(vals)
+    value = (prob.bytes() / secs / 1e9) if unit == "GB/s" else (prob.flops() / secs / 1e12)
+    line = {"metric": METRIC, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": secs * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "impl": "reference",
+            "config": {"workload": args.workload, **shape_config(prob)},
+            "cpu_baseline": {"value": value, "unit": unit, "cores": vals[0]["cores"],
+                             "kind": "oracle", "sample": vals[0]["sample"]},
+            "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def shape_config(prob):
+    c = {"layout": prob.layout, "N": prob.N, "K": prob.K}
+    if prob.layout == "dense":
+        c["M"] = prob.M
+    elif prob.layout == "contiguous":
+        c.update(G=prob.G, M_total=prob.M, valid_rows=prob.valid_rows())
+    else:
+        c.update(G=prob.G, Mmax=prob.M, valid_rows=prob.valid_rows())
+    return c
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+
+    import torch
+    import torch.distributed as dist
+    from datetime import timedelta
+    if world > 1:
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        prob, ms, e2e_ms, h2d, d2h, clocks = run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            dist.destroy_process_group()
+    if rank != 0:
+        return 0
+    unit = UNIT[args.workload]
+    value = metric_value(prob, unit, ms, world)
+    peaks, peak_src = measured_peaks()
+    if unit == "GB/s":
+        bound, peak, runit = "hbm", peaks["hbm_gbs"], "GB/s"
+        achieved = prob.bytes() / (ms * 1e-3) / 1e9
+    else:
+        bound, runit = "tensor", "TFLOP/s"
+        peak = 2.0 * peaks["bf16_tflops"]          # FP8 dense = 2 x BF16 dense (nominal ratio)
+        achieved = prob.flops() / (ms * 1e-3) / 1e12
+    pages = PAGES_NUMBER.get(args.workload)
+    line = {
+        "metric": METRIC, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": (value / pages[0]) if pages and pages[1] == unit else None,
+        "dtype": "e4m3 (f32 accumulate, bf16 out)", "data": "synthetic",
+        "config": {"workload": args.workload, **shape_config(prob),
+                   "l2": "flushed before every step (512 MB write)",
+                   "tflops": prob.flops() / (ms * 1e-3) / 1e12,
+                   "gbps": prob.bytes() / (ms * 1e-3) / 1e9},
+        "roofline": {"bound": bound, "achieved": achieved, "peak": peak, "unit": runit,
+                     "frac": achieved / peak, "traffic": profiled_traffic(args.workload),
+                     "peak_source": f"{peak_src} ({'hbm_gbs' if bound == 'hbm' else '2 x bf16_tflops'})"},
+        "e2e": {"value": metric_value(prob, unit, e2e_ms, world), "unit": unit,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": args.steps,
+        "clocks": clocks,
+    }
+    if not args.no_cpu_baseline and world == 1:
+        cb = cpu_baseline(prob, unit)
+        cb.pop("seconds_per_step", None)
+        line["cpu_baseline"] = cb
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

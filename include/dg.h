@@ -1,0 +1,151 @@
+/*
+ * dg.h -- C ABI of the B200 (sm_100a) FP8 block-scaled NT GEMM library.
+ *
+ * The operation (DeepGEMM pages: page 2 "技术特性" -- FP8 GEMM with
+ * fine-grained scaling, each K-block's tensor-core sum promoted into an FP32
+ * accumulator on CUDA cores; page 3 "核心功能" -- "fp8_gemm_nt", block-wise
+ * scaling, m-grouped GEMMs):
+ *
+ *   D[m,n] = sum_kb  sA[m,kb] * sB[n/128,kb] * sum_{k in block kb} A[m,k] * B[n,k]
+ *
+ * promoted to FP32 per 128-wide K-block and stored as BF16 (round to nearest
+ * even).  "NT": A [M,K] and B [N,K] are both K-major, D = A * B^T.
+ *
+ * Common conventions for every GEMM entry point:
+ *   - All pointers are DEVICE memory owned by the caller, 16-byte aligned.
+ *     The library allocates nothing and keeps no reference after the call
+ *     returns; the caller keeps the buffers alive until the stream work ends.
+ *   - E4M3 bytes are OCP FP8 E4M3 ("fn": no infinities, 0x7F/0xFF are NaN,
+ *     largest finite 448).
+ *   - KB = K / 128 and NB = ceil(N / 128).
+ *   - sfa ("MN-major"): the scale of row r for K-block kb is
+ *     sfa[kb * ld_sfa + r]; ld_sfa >= rows and ld_sfa % 4 == 0.
+ *   - sfb: the scale of weight block j (rows 128j..128j+127) for K-block kb is
+ *     sfb[j * KB + kb]; grouped calls hold one such [NB][KB] array per group,
+ *     back to back.
+ *   - d: BF16 [rows, N] row-major (row stride N elements).
+ *   - stream: a cudaStream_t passed as void* (NULL = legacy default stream).
+ *     Calls are asynchronous on it and never synchronise the host.
+ *   - Shape rules: K > 0, K % 128 == 0; N > 0, N % 16 == 0; M >= 0.
+ *   - Errors: every argument is validated before anything is enqueued; on an
+ *     error nothing is launched and d is untouched.  DG_ERR_CUDA reports a
+ *     failed launch or a CUDA runtime error (text via dg_last_cuda_error()).
+ *     A kernel that gives up on a bounded wait records DG_ERR_TIMEOUT in the
+ *     device status word (dg_get_device_status) instead of hanging.
+ *   - Thread safety: calls on different streams may run concurrently.
+ */
+#ifndef DG_H_
+#define DG_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define DG_API __attribute__((visibility("default")))
+#else
+#define DG_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    DG_SUCCESS = 0,
+    DG_ERR_INVALID_VALUE = 1,      /* null pointer, negative size, bad index table */
+    DG_ERR_MISALIGNED = 2,         /* pointer or leading dimension not 16-byte aligned */
+    DG_ERR_UNSUPPORTED_SHAPE = 3,  /* K % 128, N % 16, or a size beyond the limits */
+    DG_ERR_UNSUPPORTED_DEVICE = 4, /* no CUDA device, or not compute capability 10.0 */
+    DG_ERR_CUDA = 5,               /* CUDA runtime / launch failure */
+    DG_ERR_TIMEOUT = 6             /* a kernel's bounded wait ran out (device status) */
+} dg_status_t;
+
+/*
+ * Dense GEMM (page 3 "核心功能" / "快速开始": fp8_gemm_nt).
+ *   a   [M, K] E4M3;  sfa [KB, ld_sfa] FP32, ld_sfa >= M
+ *   b   [N, K] E4M3;  sfb [NB, KB] FP32
+ *   d   [M, N] BF16, fully written.
+ * M == 0 is a no-op.
+ */
+DG_API dg_status_t dg_fp8_gemm_nt(const uint8_t *a, const float *sfa, int ld_sfa,
+                           const uint8_t *b, const float *sfb,
+                           void *d, int M, int N, int K, void *stream);
+
+/*
+ * M-grouped GEMM, contiguous layout (page 2 "MoE模型专属优化"; page 5 "02",
+ * prefill).  The rows of all groups are packed back to back in a; each
+ * group's rows are padded to a multiple of
+ * dg_get_m_alignment_for_contiguous_layout() (128).
+ *   a         [M_total, K] E4M3;  sfa [KB, ld_sfa] FP32, ld_sfa >= M_total
+ *   b         [G, N, K] E4M3;     sfb [G, NB, KB] FP32
+ *   d         [M_total, N] BF16
+ *   m_indices [M_total] int32 on the device: the group of each row, -1 for
+ *             padding.  Precondition: the rows of each 128-row block carry
+ *             one group index or -1, and the block's first row is not -1
+ *             unless the whole block is padding (a block whose first row is
+ *             -1 is skipped).  Outputs of padding rows are unspecified (they
+ *             may be written).  An index >= G makes the kernel skip the block
+ *             and record DG_ERR_INVALID_VALUE in the device status word.
+ * M_total % 128 == 0; M_total == 0 is a no-op.
+ */
+DG_API dg_status_t dg_m_grouped_fp8_gemm_nt_contiguous(const uint8_t *a, const float *sfa, int ld_sfa,
+                                                const uint8_t *b, const float *sfb,
+                                                void *d, const int32_t *m_indices,
+                                                int M_total, int N, int K, int G,
+                                                void *stream);
+
+/*
+ * M-grouped GEMM, masked layout (page 2 "MoE模型专属优化"; page 5 "02",
+ * decode): a fixed [G, Mmax, K] buffer and a per-group valid-row count that
+ * only the device reads, so the call works unchanged inside a CUDA graph.
+ *   a        [G, Mmax, K] E4M3;   sfa [G, KB, ld_sfa] FP32, ld_sfa >= Mmax
+ *   b        [G, N, K] E4M3;      sfb [G, NB, KB] FP32
+ *   d        [G, Mmax, N] BF16
+ *   masked_m [G] int32 on the device, 0 <= masked_m[g] <= Mmax.
+ * Rows m < masked_m[g] of group g are computed; rows >= masked_m[g] of d are
+ * never written (bit-for-bit untouched).  Groups with masked_m[g] == 0 read
+ * nothing.  A count outside [0, Mmax] is clamped and recorded as
+ * DG_ERR_INVALID_VALUE in the device status word.  G <= 1024.
+ */
+DG_API dg_status_t dg_m_grouped_fp8_gemm_nt_masked(const uint8_t *a, const float *sfa, int ld_sfa,
+                                            const uint8_t *b, const float *sfb,
+                                            void *d, const int32_t *masked_m,
+                                            int G, int Mmax, int N, int K, void *stream);
+
+/* Row alignment of the contiguous layout (page 2 "MoE模型专属优化":
+ * get_m_alignment_for_contiguous_layout).  Returns 128. */
+DG_API int dg_get_m_alignment_for_contiguous_layout(void);
+
+/* Smallest count >= n whose size n * elem_bytes is a multiple of 16 bytes,
+ * the TMA alignment (page 2 "快速实践指南": get_tma_aligned_size).
+ * elem_bytes must divide 16 (1, 2, 4, 8, 16); otherwise returns 0. */
+DG_API size_t dg_get_tma_aligned_size(size_t n, size_t elem_bytes);
+
+/* Reads the current device's status word, which kernels set when a bounded
+ * wait runs out (DG_ERR_TIMEOUT) or a device-side index is out of range
+ * (DG_ERR_INVALID_VALUE).  Synchronises the device.  *code receives the raw
+ * word (0 = clean; low 8 bits = dg_status_t, upper bits = where).  When
+ * clear != 0 the word is reset to 0 afterwards. */
+DG_API dg_status_t dg_get_device_status(int *code, int clear);
+
+/* Static text for a status code. */
+DG_API const char *dg_status_string(dg_status_t status);
+
+/* Text of the last CUDA error seen by this library on the calling thread
+ * (empty string if none). */
+DG_API const char *dg_last_cuda_error(void);
+
+/* Test hook, not part of the GEMM contract (the pages have no counterpart):
+ * kernels launched afterwards by this process run with the given debug flags.
+ * Flag 1 makes the producer warp issue no loads, so the consumers' bounded
+ * waits run out and the kernel records DG_ERR_TIMEOUT in the device status
+ * word and returns instead of hanging.  0 restores normal operation.  The
+ * wait limit in clock cycles comes from the environment variable
+ * DG_WAIT_TIMEOUT_CYCLES, read once (default 2^32). */
+DG_API void dg_debug_set_flags(int flags);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DG_H_ */

@@ -1,0 +1,173 @@
+"""Python binding of the B200 FP8 block-scaled NT GEMM library (``_dg.so``).
+
+Argument marshalling only: every function below checks dtypes and shapes of
+torch CUDA tensors, reads their raw pointers and calls the C function of the
+same name declared in ``include/dg.h``.  All arithmetic runs in the CUDA
+kernels of ``_dg.so``.  There is no fallback: if the shared library is missing
+or fails to load, importing the library handle raises.
+
+Storage formats (see ``include/dg.h``): A/B are uint8 E4M3 bytes, K-major;
+sfa is float32 [KB, ld_sfa] ("MN-major"; [G, KB, ld_sfa] for the masked
+layout); sfb is float32 [G, NB, KB]; D is bfloat16.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+from typing import Optional
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "_dg.so")
+HEADER = os.path.join(os.path.dirname(_HERE), "include", "dg.h")
+
+DG_SUCCESS = 0
+STATUS_NAMES = {0: "DG_SUCCESS", 1: "DG_ERR_INVALID_VALUE", 2: "DG_ERR_MISALIGNED",
+                3: "DG_ERR_UNSUPPORTED_SHAPE", 4: "DG_ERR_UNSUPPORTED_DEVICE",
+                5: "DG_ERR_CUDA", 6: "DG_ERR_TIMEOUT"}
+
+_lib = None
+
+
+class DGError(RuntimeError):
+    def __init__(self, status: int, where: str, detail: str = ""):
+        self.status = status
+        msg = f"{where}: {STATUS_NAMES.get(status, status)}"
+        if detail:
+            msg += f" ({detail})"
+        super().__init__(msg)
+
+
+def exported_names():
+    """Names of the functions that include/dg.h declares."""
+    text = open(HEADER).read()
+    return re.findall(r"DG_API\s+[\w\s\*]+?\b(dg_\w+)\s*\(", text)
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded C library; raises if it was not built."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with "
+                          "`python -m moe_grouped_gemm_fp32_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    P, I = ctypes.c_void_p, ctypes.c_int
+    L.dg_fp8_gemm_nt.argtypes = [P, P, I, P, P, P, I, I, I, P]
+    L.dg_m_grouped_fp8_gemm_nt_contiguous.argtypes = [P, P, I, P, P, P, P, I, I, I, I, P]
+    L.dg_m_grouped_fp8_gemm_nt_masked.argtypes = [P, P, I, P, P, P, P, I, I, I, I, P]
+    for f in ("dg_fp8_gemm_nt", "dg_m_grouped_fp8_gemm_nt_contiguous",
+              "dg_m_grouped_fp8_gemm_nt_masked"):
+        getattr(L, f).restype = I
+    L.dg_get_m_alignment_for_contiguous_layout.argtypes = []
+    L.dg_get_m_alignment_for_contiguous_layout.restype = I
+    L.dg_get_tma_aligned_size.argtypes = [ctypes.c_size_t, ctypes.c_size_t]
+    L.dg_get_tma_aligned_size.restype = ctypes.c_size_t
+    L.dg_get_device_status.argtypes = [ctypes.POINTER(I), I]
+    L.dg_get_device_status.restype = I
+    L.dg_status_string.argtypes = [I]
+    L.dg_status_string.restype = ctypes.c_char_p
+    L.dg_last_cuda_error.argtypes = []
+    L.dg_last_cuda_error.restype = ctypes.c_char_p
+    L.dg_debug_set_flags.argtypes = [I]
+    L.dg_debug_set_flags.restype = None
+    _lib = L
+    return L
+
+
+def _check(status: int, where: str):
+    if status != DG_SUCCESS:
+        detail = lib().dg_last_cuda_error().decode() if status == 5 else ""
+        raise DGError(status, where, detail)
+
+
+def _stream_handle(stream) -> Optional[int]:
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream
+
+
+def _req(t, dtype, name, ndim=None):
+    import torch
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if ndim is not None and t.dim() not in ((ndim,) if isinstance(ndim, int) else ndim):
+        raise ValueError(f"{name} has {t.dim()} dims")
+    return t.data_ptr()
+
+
+# --------------------------------------------------------------------------- GEMMs
+def dg_fp8_gemm_nt(a, sfa, b, sfb, d, stream=None):
+    """D[M,N] (bf16) = block-scaled A[M,K] * B[N,K]^T.
+
+    a uint8 [M,K]; sfa float32 [KB, ld_sfa]; b uint8 [N,K] (or [1,N,K]);
+    sfb float32 [NB,KB] (or [1,NB,KB]); d bfloat16 [M,N]."""
+    import torch
+    M, K = a.shape
+    N = b.shape[-2]
+    ld = sfa.shape[-1]
+    st = lib().dg_fp8_gemm_nt(_req(a, torch.uint8, "a", 2), _req(sfa, torch.float32, "sfa", 2), ld,
+                              _req(b, torch.uint8, "b", (2, 3)), _req(sfb, torch.float32, "sfb", (2, 3)),
+                              _req(d, torch.bfloat16, "d", 2), M, N, K, _stream_handle(stream))
+    _check(st, "dg_fp8_gemm_nt")
+    return d
+
+
+def dg_m_grouped_fp8_gemm_nt_contiguous(a, sfa, b, sfb, d, m_indices, stream=None):
+    """Contiguous M-grouped GEMM.  a uint8 [M_total,K]; b uint8 [G,N,K];
+    sfb float32 [G,NB,KB]; d bfloat16 [M_total,N]; m_indices int32 [M_total]."""
+    import torch
+    M_total, K = a.shape
+    G, N, _ = b.shape
+    st = lib().dg_m_grouped_fp8_gemm_nt_contiguous(
+        _req(a, torch.uint8, "a", 2), _req(sfa, torch.float32, "sfa", 2), sfa.shape[-1],
+        _req(b, torch.uint8, "b", 3), _req(sfb, torch.float32, "sfb", 3),
+        _req(d, torch.bfloat16, "d", 2), _req(m_indices, torch.int32, "m_indices", 1),
+        M_total, N, K, G, _stream_handle(stream))
+    _check(st, "dg_m_grouped_fp8_gemm_nt_contiguous")
+    return d
+
+
+def dg_m_grouped_fp8_gemm_nt_masked(a, sfa, b, sfb, d, masked_m, stream=None):
+    """Masked M-grouped GEMM.  a uint8 [G,Mmax,K]; sfa float32 [G,KB,ld_sfa];
+    b uint8 [G,N,K]; sfb float32 [G,NB,KB]; d bfloat16 [G,Mmax,N];
+    masked_m int32 [G] (device).  Rows >= masked_m[g] of d are not written."""
+    import torch
+    G, Mmax, K = a.shape
+    N = b.shape[1]
+    st = lib().dg_m_grouped_fp8_gemm_nt_masked(
+        _req(a, torch.uint8, "a", 3), _req(sfa, torch.float32, "sfa", 3), sfa.shape[-1],
+        _req(b, torch.uint8, "b", 3), _req(sfb, torch.float32, "sfb", 3),
+        _req(d, torch.bfloat16, "d", 3), _req(masked_m, torch.int32, "masked_m", 1),
+        G, Mmax, N, K, _stream_handle(stream))
+    _check(st, "dg_m_grouped_fp8_gemm_nt_masked")
+    return d
+
+
+# --------------------------------------------------------------------------- helpers
+def dg_get_m_alignment_for_contiguous_layout() -> int:
+    return lib().dg_get_m_alignment_for_contiguous_layout()
+
+
+def dg_get_tma_aligned_size(n: int, elem_bytes: int = 4) -> int:
+    return lib().dg_get_tma_aligned_size(n, elem_bytes)
+
+
+def dg_get_device_status(clear: bool = True) -> int:
+    code = ctypes.c_int(0)
+    _check(lib().dg_get_device_status(ctypes.byref(code), int(clear)), "dg_get_device_status")
+    return code.value
+
+
+def dg_status_string(status: int) -> str:
+    return lib().dg_status_string(status).decode()
+
+
+def dg_debug_set_flags(flags: int) -> None:
+    lib().dg_debug_set_flags(flags)

@@ -1,0 +1,395 @@
+// dg_api.cu -- host side of the C ABI declared in include/dg.h: argument
+// validation, TMA descriptor encoding, tile-configuration choice and kernel
+// launch.  Nothing here synchronises the host (except dg_get_device_status)
+// or allocates memory.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+
+#include "dg.h"
+#include "gemm_kernel.cuh"
+
+namespace {
+
+__device__ unsigned g_dg_status = 0u;
+
+thread_local char t_last_cuda_error[256] = "";
+
+dg_status_t cuda_fail(cudaError_t e, const char *what) {
+    std::snprintf(t_last_cuda_error, sizeof(t_last_cuda_error), "%s: %s", what,
+                  cudaGetErrorString(e));
+    return DG_ERR_CUDA;
+}
+
+// ------------------------------------------------------------------ device info
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+    bool ready = false;
+    bool supported = false;
+    int num_sms = 0;
+    unsigned *status = nullptr;   // device address of g_dg_status
+};
+
+DeviceInfo g_devices[kMaxDevices];
+std::mutex g_mutex;
+
+dg_status_t device_info(const DeviceInfo **out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return DG_ERR_UNSUPPORTED_DEVICE;
+    }
+    if (dev < 0 || dev >= kMaxDevices) return DG_ERR_UNSUPPORTED_DEVICE;
+    std::lock_guard<std::mutex> lock(g_mutex);
+    DeviceInfo &info = g_devices[dev];
+    if (!info.ready) {
+        int major = 0, minor = 0, sms = 0;
+        if ((e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev)) != cudaSuccess ||
+            (e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev)) != cudaSuccess ||
+            (e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+            return cuda_fail(e, "cudaDeviceGetAttribute");
+        info.supported = (major == 10 && minor == 0);
+        info.num_sms = sms;
+        if (info.supported) {
+            void *addr = nullptr;
+            if ((e = cudaGetSymbolAddress(&addr, g_dg_status)) != cudaSuccess)
+                return cuda_fail(e, "cudaGetSymbolAddress(status)");
+            info.status = static_cast<unsigned *>(addr);
+        }
+        info.ready = true;
+    }
+    if (!info.supported) return DG_ERR_UNSUPPORTED_DEVICE;
+    *out = &info;
+    return DG_SUCCESS;
+}
+
+// ------------------------------------------------------------------ tensor maps
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+        else
+            cudaGetLastError();
+    });
+    return fn;
+}
+
+// 3-D uint8 tensor {K, rows, groups} (K innermost), box {128, box_rows, 1},
+// 128-byte swizzle, zero fill out of bounds.
+dg_status_t make_map(CUtensorMap *m, const void *base, long long K, long long rows,
+                     long long groups, int box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) {
+        std::snprintf(t_last_cuda_error, sizeof(t_last_cuda_error),
+                      "cuTensorMapEncodeTiled entry point unavailable");
+        return DG_ERR_CUDA;
+    }
+    cuuint64_t dims[3] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows),
+                          static_cast<cuuint64_t>(groups)};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(K * rows)};
+    cuuint32_t box[3] = {static_cast<cuuint32_t>(dg::kBlockK), static_cast<cuuint32_t>(box_rows), 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(base), dims, strides,
+                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        std::snprintf(t_last_cuda_error, sizeof(t_last_cuda_error),
+                      "cuTensorMapEncodeTiled failed (CUresult %d)", static_cast<int>(r));
+        return DG_ERR_CUDA;
+    }
+    return DG_SUCCESS;
+}
+
+// ------------------------------------------------------------------ validation
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+dg_status_t check_common(const void *a, const float *sfa, int ld_sfa, const void *b,
+                         const float *sfb, const void *d, int rows, int N, int K) {
+    if (!a || !sfa || !b || !sfb || !d) return DG_ERR_INVALID_VALUE;
+    if (rows < 0 || N <= 0 || K <= 0) return DG_ERR_INVALID_VALUE;
+    if (K % dg::kBlockK != 0 || N % 16 != 0) return DG_ERR_UNSUPPORTED_SHAPE;
+    if (ld_sfa < rows || ld_sfa <= 0) return DG_ERR_INVALID_VALUE;
+    if (ld_sfa % 4 != 0) return DG_ERR_MISALIGNED;
+    if (!aligned16(a) || !aligned16(b) || !aligned16(d) || !aligned16(sfa) || !aligned16(sfb))
+        return DG_ERR_MISALIGNED;
+    // TMA coordinates and element offsets stay within 32-bit ranges
+    if (static_cast<long long>(K) > (1LL << 30) || N > (1 << 30)) return DG_ERR_UNSUPPORTED_SHAPE;
+    return DG_SUCCESS;
+}
+
+long long timeout_cycles() {
+    static long long v = [] {
+        const char *s = std::getenv("DG_WAIT_TIMEOUT_CYCLES");
+        long long x = s ? std::atoll(s) : 0;
+        return x > 0 ? x : (1LL << 32);   // ~2 s at 2 GHz; legitimate waits are micro- to milliseconds
+    }();
+    return v;
+}
+
+int g_debug_flags = 0;
+
+// ------------------------------------------------------------------ launch
+template <int kBN, bool kSwap, int kStages, int kLayout>
+dg_status_t launch(const CUtensorMap &ma, const CUtensorMap &mb, const dg::Params &p, int grid_x,
+                   int grid_y, int cluster_x, cudaStream_t stream) {
+    using L = dg::SmemLayout<kBN, kStages>;
+    auto kernel = dg::fp8_gemm_kernel<kBN, kSwap, kStages, kLayout>;
+    static bool attr_done[kMaxDevices] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (!attr_done[dev]) {
+        cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             L::kAlloc);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+        attr_done[dev] = true;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid_x, grid_y, 1);
+    cfg.blockDim = dim3(dg::kNumThreads, 1, 1);
+    cfg.dynamicSmemBytes = L::kAlloc;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    cfg.attrs = attr;
+    cfg.numAttrs = 0;
+    if (cluster_x > 1) {
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = cluster_x;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.numAttrs = 1;
+    }
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, ma, mb, p);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaLaunchKernelEx");
+    return DG_SUCCESS;
+}
+
+// How many clusters of `cluster_x` CTAs of this kernel can be resident at once
+// (cached per device and cluster size).  0 if the query fails.
+template <int kBN, bool kSwap, int kStages, int kLayout>
+int max_active_clusters(int cluster_x) {
+    using L = dg::SmemLayout<kBN, kStages>;
+    auto kernel = dg::fp8_gemm_kernel<kBN, kSwap, kStages, kLayout>;
+    static int cache[kMaxDevices][9] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (cluster_x < 1 || cluster_x > 8) return 0;
+    if (cache[dev][cluster_x]) return cache[dev][cluster_x];
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc) !=
+        cudaSuccess) {
+        cudaGetLastError();
+        return 0;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(cluster_x, 1, 1);
+    cfg.blockDim = dim3(dg::kNumThreads, 1, 1);
+    cfg.dynamicSmemBytes = L::kAlloc;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = cluster_x;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, kernel, &cfg) != cudaSuccess) {
+        cudaGetLastError();
+        return 0;
+    }
+    cache[dev][cluster_x] = n;
+    return n;
+}
+
+// Split-K factor for swap-mode tiles: the largest power of two <= 8 such that
+// every cluster of the grid is resident at once (one wave), each CTA keeps at
+// least two K-blocks, and the CTAs fit on the SMs.  DG_SPLIT_K overrides it
+// (tuning sweeps).
+template <int kBN, int kLayout>
+int choose_split(int tiles, int num_kb, int num_sms) {
+    static int forced = [] {
+        const char *s = std::getenv("DG_SPLIT_K");
+        return s ? std::atoi(s) : 0;
+    }();
+    if (forced == 1 || forced == 2 || forced == 4 || forced == 8)
+        return num_kb >= forced ? forced : 1;
+    for (int split = 8; split >= 2; split /= 2) {
+        if (tiles * split > num_sms || num_kb < 2 * split) continue;
+        constexpr int kStages = kBN == 64 ? 8 : (kBN == 128 ? 6 : 4);
+        if (max_active_clusters<kBN, true, kStages, kLayout>(split) >= tiles) return split;
+    }
+    return 1;
+}
+
+dg::Params base_params(const float *sfa, int ld_sfa, const float *sfb, void *d, int rows, int N,
+                       int K, int G, const DeviceInfo *info) {
+    dg::Params p = {};
+    p.sfa = sfa;
+    p.sfb = sfb;
+    p.d = static_cast<__nv_bfloat16 *>(d);
+    p.status = info->status;
+    p.timeout_cycles = timeout_cycles();
+    p.ld_sfa = ld_sfa;
+    p.M = rows;
+    p.N = N;
+    p.K = K;
+    p.G = G;
+    p.num_kb = K / dg::kBlockK;
+    p.num_nb = (N + 127) / 128;
+    p.split = 1;
+    p.debug_flags = g_debug_flags;
+    return p;
+}
+
+
+}  // namespace
+
+// ==================================================================== C ABI
+extern "C" {
+
+dg_status_t dg_fp8_gemm_nt(const uint8_t *a, const float *sfa, int ld_sfa, const uint8_t *b,
+                           const float *sfb, void *d, int M, int N, int K, void *stream) {
+    dg_status_t st = check_common(a, sfa, ld_sfa, b, sfb, d, M, N, K);
+    if (st != DG_SUCCESS) return st;
+    const DeviceInfo *info = nullptr;
+    if ((st = device_info(&info)) != DG_SUCCESS) return st;
+    if (M == 0) return DG_SUCCESS;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    dg::Params p = base_params(sfa, ld_sfa, sfb, d, M, N, K, 1, info);
+    CUtensorMap ma, mb;
+    if (M <= 256) {
+        // swap-AB: weights on the 128 TMEM lanes, the few tokens on the MMA's N side
+        const int bn = M <= 64 ? 64 : (M <= 128 ? 128 : 256);
+        const int tiles = ((N + 127) / 128) * ((M + bn - 1) / bn);
+        p.split = bn == 64    ? choose_split<64, dg::kDense>(tiles, p.num_kb, info->num_sms)
+                  : bn == 128 ? choose_split<128, dg::kDense>(tiles, p.num_kb, info->num_sms)
+                              : choose_split<256, dg::kDense>(tiles, p.num_kb, info->num_sms);
+        if ((st = make_map(&mb, b, K, N, 1, 128)) != DG_SUCCESS) return st;
+        if ((st = make_map(&ma, a, K, M, 1, bn)) != DG_SUCCESS) return st;
+        const int gx = p.split > 1 ? p.split : (tiles < info->num_sms ? tiles : info->num_sms);
+        const int gy = p.split > 1 ? tiles : 1;
+        if (bn == 64) return launch<64, true, 8, dg::kDense>(ma, mb, p, gx, gy, p.split, s);
+        if (bn == 128) return launch<128, true, 6, dg::kDense>(ma, mb, p, gx, gy, p.split, s);
+        return launch<256, true, 4, dg::kDense>(ma, mb, p, gx, gy, p.split, s);
+    }
+    const int bn = N <= 128 ? 128 : 256;
+    const int tiles = ((M + 127) / 128) * ((N + bn - 1) / bn);
+    const int grid = tiles < info->num_sms ? tiles : info->num_sms;
+    if ((st = make_map(&ma, a, K, M, 1, 128)) != DG_SUCCESS) return st;
+    if ((st = make_map(&mb, b, K, N, 1, bn)) != DG_SUCCESS) return st;
+    if (bn == 128) return launch<128, false, 6, dg::kDense>(ma, mb, p, grid, 1, 1, s);
+    return launch<256, false, 4, dg::kDense>(ma, mb, p, grid, 1, 1, s);
+}
+
+dg_status_t dg_m_grouped_fp8_gemm_nt_contiguous(const uint8_t *a, const float *sfa, int ld_sfa,
+                                                const uint8_t *b, const float *sfb, void *d,
+                                                const int32_t *m_indices, int M_total, int N,
+                                                int K, int G, void *stream) {
+    dg_status_t st = check_common(a, sfa, ld_sfa, b, sfb, d, M_total, N, K);
+    if (st != DG_SUCCESS) return st;
+    if (!m_indices || G <= 0) return DG_ERR_INVALID_VALUE;
+    if (M_total % 128 != 0) return DG_ERR_UNSUPPORTED_SHAPE;
+    const DeviceInfo *info = nullptr;
+    if ((st = device_info(&info)) != DG_SUCCESS) return st;
+    if (M_total == 0) return DG_SUCCESS;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    dg::Params p = base_params(sfa, ld_sfa, sfb, d, M_total, N, K, G, info);
+    p.m_indices = m_indices;
+    const int bn = N <= 128 ? 128 : 256;
+    const int tiles = (M_total / 128) * ((N + bn - 1) / bn);
+    const int grid = tiles < info->num_sms ? tiles : info->num_sms;
+    CUtensorMap ma, mb;
+    if ((st = make_map(&ma, a, K, M_total, 1, 128)) != DG_SUCCESS) return st;
+    if ((st = make_map(&mb, b, K, N, G, bn)) != DG_SUCCESS) return st;
+    if (bn == 128) return launch<128, false, 6, dg::kContiguous>(ma, mb, p, grid, 1, 1, s);
+    return launch<256, false, 4, dg::kContiguous>(ma, mb, p, grid, 1, 1, s);
+}
+
+dg_status_t dg_m_grouped_fp8_gemm_nt_masked(const uint8_t *a, const float *sfa, int ld_sfa,
+                                            const uint8_t *b, const float *sfb, void *d,
+                                            const int32_t *masked_m, int G, int Mmax, int N,
+                                            int K, void *stream) {
+    dg_status_t st = check_common(a, sfa, ld_sfa, b, sfb, d, Mmax, N, K);
+    if (st != DG_SUCCESS) return st;
+    if (!masked_m || G <= 0) return DG_ERR_INVALID_VALUE;
+    if (G > dg::kMaxGroups) return DG_ERR_UNSUPPORTED_SHAPE;
+    const DeviceInfo *info = nullptr;
+    if ((st = device_info(&info)) != DG_SUCCESS) return st;
+    if (Mmax == 0) return DG_SUCCESS;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    dg::Params p = base_params(sfa, ld_sfa, sfb, d, Mmax, N, K, G, info);
+    p.masked_m = masked_m;
+    const int bn = Mmax <= 64 ? 64 : (Mmax <= 128 ? 128 : 256);
+    CUtensorMap ma, mb;
+    if ((st = make_map(&mb, b, K, N, G, 128)) != DG_SUCCESS) return st;
+    if ((st = make_map(&ma, a, K, Mmax, G, bn)) != DG_SUCCESS) return st;
+    const int grid = info->num_sms;   // the tile count lives on the device
+    if (bn == 64) return launch<64, true, 8, dg::kMasked>(ma, mb, p, grid, 1, 1, s);
+    if (bn == 128) return launch<128, true, 6, dg::kMasked>(ma, mb, p, grid, 1, 1, s);
+    return launch<256, true, 4, dg::kMasked>(ma, mb, p, grid, 1, 1, s);
+}
+
+int dg_get_m_alignment_for_contiguous_layout(void) { return 128; }
+
+size_t dg_get_tma_aligned_size(size_t n, size_t elem_bytes) {
+    if (elem_bytes == 0 || elem_bytes > 16 || 16 % elem_bytes != 0) return 0;
+    const size_t q = 16 / elem_bytes;
+    return (n + q - 1) / q * q;
+}
+
+dg_status_t dg_get_device_status(int *code, int clear) {
+    if (!code) return DG_ERR_INVALID_VALUE;
+    const DeviceInfo *info = nullptr;
+    dg_status_t st = device_info(&info);
+    if (st != DG_SUCCESS) return st;
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
+    unsigned v = 0;
+    if ((e = cudaMemcpyFromSymbol(&v, g_dg_status, sizeof(v))) != cudaSuccess)
+        return cuda_fail(e, "cudaMemcpyFromSymbol(status)");
+    *code = static_cast<int>(v);
+    if (clear) {
+        const unsigned zero = 0;
+        if ((e = cudaMemcpyToSymbol(g_dg_status, &zero, sizeof(zero))) != cudaSuccess)
+            return cuda_fail(e, "cudaMemcpyToSymbol(status)");
+    }
+    return DG_SUCCESS;
+}
+
+const char *dg_status_string(dg_status_t status) {
+    switch (status) {
+        case DG_SUCCESS: return "success";
+        case DG_ERR_INVALID_VALUE: return "invalid value";
+        case DG_ERR_MISALIGNED: return "pointer or leading dimension not 16-byte aligned";
+        case DG_ERR_UNSUPPORTED_SHAPE: return "unsupported shape";
+        case DG_ERR_UNSUPPORTED_DEVICE: return "unsupported device (needs compute capability 10.0)";
+        case DG_ERR_CUDA: return "CUDA error";
+        case DG_ERR_TIMEOUT: return "a kernel wait timed out";
+    }
+    return "unknown status";
+}
+
+const char *dg_last_cuda_error(void) { return t_last_cuda_error; }
+
+// Test hook (not part of the GEMM contract): kernels launched afterwards on
+// this process run with the given debug flags.  Flag 1 makes the producer warp
+// issue no loads, so the consumers' bounded waits run out and the kernel
+// reports DG_ERR_TIMEOUT through the status word instead of hanging.
+void dg_debug_set_flags(int flags) { g_debug_flags = flags; }
+
+}  // extern "C"

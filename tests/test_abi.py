@@ -1,0 +1,92 @@
+"""Host-only checks of the C ABI (no GPU needed): the shared library loads,
+exports every function include/dg.h declares, the helpers return the
+documented values, and invalid arguments are rejected before any CUDA call."""
+import ctypes
+import subprocess
+
+import pytest
+
+import moe_grouped_gemm_fp32_b200 as dg
+from moe_grouped_gemm_fp32_b200 import build as dg_build
+
+
+@pytest.fixture(scope="module")
+def L():
+    dg_build.build()
+    return dg.lib()
+
+
+def test_header_declares_the_three_gemms_and_helpers():
+    names = dg.exported_names()
+    for n in ("dg_fp8_gemm_nt", "dg_m_grouped_fp8_gemm_nt_contiguous",
+              "dg_m_grouped_fp8_gemm_nt_masked", "dg_get_m_alignment_for_contiguous_layout",
+              "dg_get_tma_aligned_size", "dg_get_device_status", "dg_status_string"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(L):
+    out = subprocess.run(["nm", "-D", "--defined-only", dg.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if line.strip()}
+    for n in dg.exported_names():
+        assert n in exported, n
+        assert hasattr(L, n)
+    # nothing else with the library prefix leaks out
+    assert {e for e in exported if e.startswith("dg_")} == set(dg.exported_names())
+
+
+def test_helpers(L):
+    assert dg.dg_get_m_alignment_for_contiguous_layout() == 128
+    assert dg.dg_get_tma_aligned_size(1, 4) == 4
+    assert dg.dg_get_tma_aligned_size(64, 4) == 64
+    assert dg.dg_get_tma_aligned_size(65, 4) == 68
+    assert dg.dg_get_tma_aligned_size(17, 1) == 32
+    assert dg.dg_get_tma_aligned_size(3, 2) == 8
+    assert dg.dg_get_tma_aligned_size(5, 3) == 0
+    assert dg.dg_status_string(6) == "a kernel wait timed out"
+    assert dg.dg_status_string(0) == "success"
+
+
+FAKE = 0x10000   # a 16-byte aligned non-null address; never dereferenced on these paths
+
+
+def _dense(L, **kw):
+    args = dict(a=FAKE, sfa=FAKE, ld=64, b=FAKE, sfb=FAKE, d=FAKE, M=64, N=256, K=512)
+    args.update(kw)
+    return L.dg_fp8_gemm_nt(args["a"], args["sfa"], args["ld"], args["b"], args["sfb"],
+                            args["d"], args["M"], args["N"], args["K"], None)
+
+
+def test_dense_validation(L):
+    assert _dense(L, a=None) == 1
+    assert _dense(L, d=None) == 1
+    assert _dense(L, M=-1) == 1
+    assert _dense(L, K=100) == 3
+    assert _dense(L, K=0) == 1
+    assert _dense(L, N=200) == 3
+    assert _dense(L, ld=32) == 1            # ld_sfa < M
+    assert _dense(L, ld=66) == 2            # ld_sfa not a multiple of 4
+    assert _dense(L, a=FAKE + 8) == 2
+    assert _dense(L, sfb=FAKE + 4) == 2
+    # valid arguments on a host without a usable B200: refused as an unsupported device
+    assert _dense(L) in (4,)
+
+
+def test_grouped_validation(L):
+    c = L.dg_m_grouped_fp8_gemm_nt_contiguous
+    assert c(FAKE, FAKE, 256, FAKE, FAKE, FAKE, None, 256, 256, 512, 4, None) == 1   # m_indices
+    assert c(FAKE, FAKE, 256, FAKE, FAKE, FAKE, FAKE, 200, 256, 512, 4, None) == 3   # M_total % 128
+    assert c(FAKE, FAKE, 256, FAKE, FAKE, FAKE, FAKE, 256, 256, 512, 0, None) == 1   # G
+    m = L.dg_m_grouped_fp8_gemm_nt_masked
+    assert m(FAKE, FAKE, 256, FAKE, FAKE, FAKE, None, 4, 256, 256, 512, None) == 1   # masked_m
+    assert m(FAKE, FAKE, 256, FAKE, FAKE, FAKE, FAKE, 2000, 256, 256, 512, None) == 3  # G > 1024
+    assert m(FAKE, FAKE, 128, FAKE, FAKE, FAKE, FAKE, 4, 256, 256, 512, None) == 1   # ld < Mmax
+    assert m(FAKE, FAKE, 256, FAKE, FAKE, FAKE, FAKE, 4, 256, 256, 384, None) == 4   # no device
+
+
+def test_python_binding_rejects_cpu_tensors():
+    import torch
+    a = torch.zeros((64, 128), dtype=torch.uint8)
+    with pytest.raises(TypeError):
+        dg.dg_fp8_gemm_nt(a, torch.zeros((1, 64)), torch.zeros((128, 128), dtype=torch.uint8),
+                          torch.zeros((1, 1)), torch.zeros((64, 128), dtype=torch.bfloat16))

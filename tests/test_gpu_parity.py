@@ -1,0 +1,221 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle.
+
+Tolerance (the workload definition's): per element |D - D_ref| <= 1e-2 *
+max(1, |D_ref|) and relative Frobenius error <= 2e-3 over valid rows.
+Integer-valued cases with power-of-two scales must match bit for bit.
+Padding rows hold NaN bytes and NaN scales (a leak shows as NaN); D is
+pre-filled with a sentinel so that rows the method must not write can be
+checked bit for bit.
+"""
+import numpy as np
+import pytest
+import torch
+
+import moe_grouped_gemm_fp32_b200 as dg
+import oracle
+import workloads as W
+from gpu_util import SENTINEL, DeviceProblem, compare, to_f64, valid_mask
+
+pytestmark = [pytest.mark.gpu,
+              pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CUDA GPU")]
+
+
+@pytest.fixture(autouse=True, scope="module")
+def _clean_status():
+    from moe_grouped_gemm_fp32_b200 import build
+    build.build()
+    dg.dg_get_device_status(clear=True)
+    yield
+    assert dg.dg_get_device_status(clear=True) == 0, "a kernel recorded an error"
+
+
+def _run_full(prob, sentinel=True):
+    dp = DeviceProblem(prob)
+    if sentinel:
+        dp.fill_sentinel()
+    d = to_f64(dp.run())
+    torch.cuda.synchronize()
+    ref = oracle.solve(prob)
+    margins = compare(d, ref, valid_mask(prob))
+    return dp, d, ref, margins
+
+
+# ------------------------------------------------------------------ dense
+def test_dense_tiny():
+    _run_full(W.make_workload("dense_tiny"))
+
+
+@pytest.mark.parametrize("M", [1, 63, 64, 65, 127, 128, 129, 200, 256, 257, 300])
+def test_dense_m_sweep_with_n_tail(M):
+    # N = 2112 = 16.5 weight blocks: a half-filled last block; K = 1024 (8 K-blocks)
+    _run_full(W.make_dense(M, 2112, 1024, seed=100 + M, outliers=True))
+
+
+@pytest.mark.parametrize("M,K", [(64, 4096), (128, 4096), (16, 7168)])
+def test_dense_small_m_split_k(M, K):
+    # enough K-blocks for an 8-CTA split-K cluster
+    _run_full(W.make_dense(M, 2112, K, seed=7 + M, outliers=True))
+
+
+@pytest.mark.parametrize("M,N", [(512, 256), (384, 384), (1024, 1152)])
+def test_dense_normal_mode(M, N):
+    _run_full(W.make_dense(M, N, 1024, seed=M + N))
+
+
+def test_dense_wide_tile_n_128():
+    _run_full(W.make_dense(512, 128, 512, seed=3))
+
+
+def _exact_dense(M, N, K, seed):
+    """Operands in {-1,0,1} (sparse), power-of-two scales: every partial sum
+    and every output is exact in FP32 and representable in BF16."""
+    rng = np.random.default_rng(seed)
+    KB, NB = K // 128, (N + 127) // 128
+    ai = rng.choice([-1, 0, 0, 0, 0, 0, 0, 1], size=(M, K))
+    bi = rng.choice([-1, 0, 0, 0, 0, 0, 0, 1], size=(N, K))
+    to8 = lambda v: torch.from_numpy(v.astype(np.float32)).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    sa = np.ldexp(1.0, rng.integers(-1, 2, size=(M, KB))).astype(np.float32)
+    sb = np.ldexp(1.0, rng.integers(-1, 1, size=(NB, KB))).astype(np.float32)
+    ld = W.tma_aligned(M)
+    return W.Problem("dense", M, N, K, 1, to8(ai), W.sfa_mn_major(sa, ld), ld, to8(bi)[None], sb[None])
+
+
+@pytest.mark.parametrize("M", [32, 64, 128, 300])
+def test_dense_integer_cases_bit_exact(M):
+    prob = _exact_dense(M, 384, 512, seed=M)
+    ref = oracle.solve(prob)
+    ref_bf16 = torch.from_numpy(ref).to(torch.bfloat16)
+    assert torch.equal(ref_bf16.double(), torch.from_numpy(ref)), "case not BF16-exact"
+    d = DeviceProblem(prob).run().cpu()
+    assert torch.equal(d.view(torch.int16), ref_bf16.view(torch.int16))
+
+
+def test_dense_deterministic():
+    prob = W.make_dense(64, 2112, 4096, seed=11, outliers=True)
+    dp = DeviceProblem(prob)
+    d1 = dp.run().clone()
+    d2 = dp.run().clone()
+    assert torch.equal(d1.view(torch.int16), d2.view(torch.int16))
+
+
+# ------------------------------------------------------------------ contiguous
+@pytest.mark.parametrize("counts,N,K", [([130, 0, 700, 5], 384, 512),
+                                        ([0, 0, 1, 0], 256, 256),
+                                        ([128, 256], 2112, 512)])
+def test_contiguous(counts, N, K):
+    _run_full(W.make_contiguous(counts, N, K, seed=sum(counts) + N))
+
+
+def test_contiguous_multinomial_small():
+    _run_full(W.make_contiguous_multinomial(4, 2000, 256, 1024, seed=4))
+
+
+def test_contiguous_equals_dense_per_group():
+    prob = W.make_contiguous([200, 100, 300], 256, 512, seed=12)
+    dp = DeviceProblem(prob)
+    d = dp.run().clone()
+    for g in range(prob.G):
+        rows = np.flatnonzero(prob.m_indices == g)
+        sub = W.Problem("dense", len(rows), prob.N, prob.K, 1, prob.a[rows],
+                        W.sfa_mn_major(prob.sfa[:, rows].T.copy(), W.tma_aligned(len(rows))),
+                        W.tma_aligned(len(rows)), prob.b[g:g + 1], prob.sfb[g:g + 1])
+        dd = DeviceProblem(sub).run()
+        ref = oracle.solve(sub)
+        compare(to_f64(d[torch.from_numpy(rows).cuda()]), ref, np.ones_like(ref, bool))
+        compare(to_f64(dd), ref, np.ones_like(ref, bool))
+
+
+# ------------------------------------------------------------------ masked
+@pytest.mark.parametrize("masked_m,Mmax", [([0, 256, 1, 100, 255, 64, 65, 128], 256),
+                                           ([64, 0, 17, 63], 64),
+                                           ([128, 5, 0, 127, 64], 128),
+                                           ([0, 0, 0], 256)])
+def test_masked_rows_untouched(masked_m, Mmax):
+    prob = W.make_masked(masked_m, Mmax, 384, 512, seed=Mmax + len(masked_m))
+    dp, d, ref, _ = _run_full(prob, sentinel=True)
+    raw = dp.d.view(torch.int16).cpu().numpy()
+    for g, m in enumerate(masked_m):
+        assert (raw[g, m:] == np.int16(SENTINEL)).all(), f"group {g} rows >= {m} written"
+        assert (raw[g, :m] != np.int16(SENTINEL)).all()
+
+
+def test_masked_n_tail_large_k():
+    _run_full(W.make_masked([200, 33, 0, 256], 256, 2112, 2048, seed=21))
+
+
+def test_masked_cuda_graph_replay_reads_new_counts():
+    """The masked call reads masked_m on the device only: a captured graph
+    replayed after the counts change computes (and leaves untouched) the rows
+    the NEW counts say."""
+    prob = W.make_masked([10, 200, 0, 64], 256, 256, 512, seed=31, poison=False)
+    dp = DeviceProblem(prob)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        dp.run(s)                        # first call outside the capture
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        dp.run(s)
+    new_m = np.array([256, 0, 100, 1], np.int32)
+    dp.masked_m.copy_(torch.from_numpy(new_m))
+    dp.fill_sentinel()
+    torch.cuda.synchronize()
+    g.replay()
+    torch.cuda.synchronize()
+    prob2 = W.Problem("masked", prob.M, prob.N, prob.K, prob.G, prob.a, prob.sfa, prob.ld_sfa,
+                      prob.b, prob.sfb, masked_m=new_m)
+    compare(to_f64(dp.d), oracle.solve(prob2), valid_mask(prob2))
+    raw = dp.d.view(torch.int16).cpu().numpy()
+    for gi, m in enumerate(new_m):
+        assert (raw[gi, m:] == np.int16(SENTINEL)).all()
+    del g
+
+
+def test_masked_equals_dense_per_group():
+    prob = W.make_masked([77, 0, 256, 130], 256, 384, 1024, seed=41)
+    d = DeviceProblem(prob).run().clone()
+    for g, m in enumerate(prob.masked_m):
+        if m == 0:
+            continue
+        sub = W.Problem("dense", int(m), prob.N, prob.K, 1, prob.a[g, :m],
+                        np.ascontiguousarray(prob.sfa[g]), prob.ld_sfa, prob.b[g:g + 1], prob.sfb[g:g + 1])
+        dd = DeviceProblem(sub).run()
+        ref = oracle.solve(sub)
+        compare(to_f64(d[g, :m]), ref, np.ones_like(ref, bool))
+        compare(to_f64(dd), ref, np.ones_like(ref, bool))
+
+
+# ------------------------------------------------------------------ full-size workloads
+@pytest.mark.parametrize("name", ["dense_decode_m64", "dense_decode_m128"])
+def test_full_size_decode_full_oracle(name):
+    _run_full(W.make_workload(name))
+
+
+@pytest.mark.parametrize("name", ["dense_large", "contiguous_g4", "masked_g16"])
+def test_full_size_sampled(name):
+    prob = W.make_workload(name)
+    dp = DeviceProblem(prob)
+    dp.fill_sentinel()
+    d = to_f64(dp.run())
+    rng = np.random.default_rng(2024)
+    n = 6000
+    mask = valid_mask(prob)
+    if prob.layout == "masked":
+        grp = rng.integers(0, prob.G, n)
+        row = np.array([rng.integers(0, max(int(prob.masked_m[g]), 1)) for g in grp])
+        keep = prob.masked_m[grp] > 0
+        grp, row = grp[keep], row[keep]
+    else:
+        grp = np.zeros(n, np.int64)
+        valid_rows = np.flatnonzero(mask[:, 0])
+        row = rng.choice(valid_rows, n)
+    col = rng.integers(0, prob.N, len(row))
+    ref = oracle.points(prob, grp, row, col)
+    got = d[grp, row, col] if prob.layout == "masked" else d[row, col]
+    compare(got, ref, np.ones_like(ref, bool))
+    # properties that hold at any size: no NaN in valid rows, untouched masked rows
+    assert np.isfinite(d[mask]).all()
+    if prob.layout == "masked":
+        raw = dp.d.view(torch.int16).cpu().numpy()
+        for g, m in enumerate(prob.masked_m):
+            assert (raw[g, m:] == np.int16(SENTINEL)).all()
