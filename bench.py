@@ -21,7 +21,6 @@ import json
 import os
 import re
 import statistics
-import subprocess
 import sys
 import threading
 import time
@@ -73,59 +72,63 @@ def profiled_traffic(workload: str):
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons, sampled in the background."""
-    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
-              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
-              "clocks_event_reasons.sw_power_cap")
+    """SM clock and throttle reasons of one GPU, read through NVML every few
+    milliseconds by a background thread while the timed region runs.  Reads
+    only; no setting of the GPU is touched."""
 
-    def __init__(self, gpu_index: str):
-        self.gpu = gpu_index
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"))
+
+    def __init__(self, torch_device):
+        self.dev = torch_device
         self.samples = []
-        self.proc = None
+        self.stop_evt = threading.Event()
         self.thread = None
+        self.nvml = None
+        self.handle = None
+        self.max_mhz = None
 
     def start(self):
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "50"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-        except OSError:
-            self.proc = None
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            props = torch.cuda.get_device_properties(self.dev)
+            bus = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
+            self.handle = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.handle, pynvml.NVML_CLOCK_SM)
+            self.nvml = pynvml
+        except Exception:
+            self.nvml = None
             return
-        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread = threading.Thread(target=self._run, daemon=True)
         self.thread.start()
 
-    def _read(self):
-        for line in self.proc.stdout:
-            parts = [x.strip() for x in line.split(",")]
-            if len(parts) == 7:
-                self.samples.append(parts)
+    def _run(self):
+        nv = self.nvml
+        while not self.stop_evt.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self.handle, nv.NVML_CLOCK_SM)
+                mask = nv.nvmlDeviceGetCurrentClocksEventReasons(self.handle)
+                self.samples.append((time.perf_counter(), mhz, mask))
+            except Exception:
+                pass
+            self.stop_evt.wait(0.005)
 
     def stop(self):
-        if self.proc is not None:
-            self.proc.terminate()
-            try:
-                self.proc.wait(timeout=5)
-            except subprocess.TimeoutExpired:
-                self.proc.kill()
-        if self.thread is not None:
-            self.thread.join(timeout=5)
+        if self.thread is None:
+            return None
+        self.stop_evt.set()
+        self.thread.join(timeout=5)
         if not self.samples:
             return None
-        def num(x):
-            try:
-                return float(x)
-            except ValueError:
-                return None
-        sm = [num(s[0]) for s in self.samples if num(s[0]) is not None]
-        mx = [num(s[1]) for s in self.samples if num(s[1]) is not None]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for s in self.samples for i in range(4)
-                          if s[3 + i].lower() in ("active", "1")})
-        return {"sm_mhz": statistics.median(sm) if sm else None,
-                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
-                "samples": len(self.samples)}
+        nv = self.nvml
+        reasons = sorted({name for _, _, mask in self.samples for name, attr in self.REASONS
+                          if mask & getattr(nv, attr, 0)})
+        return {"sm_mhz": statistics.median(m for _, m, _ in self.samples),
+                "sm_max_mhz": self.max_mhz, "reasons": reasons, "samples": len(self.samples)}
 
 
 # ----------------------------------------------------------------------------- our arm
@@ -180,8 +183,7 @@ def run_ours(args, rank, world, local_rank):
             dist.barrier(device_ids=[local_rank])
         torch.cuda.synchronize(dev)
 
-    visible = [v.strip() for v in os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",") if v.strip()]
-    sampler = ClockSampler(visible[local_rank] if local_rank < len(visible) else str(local_rank))
+    sampler = ClockSampler(dev)
     # ---- device-resident timing
     for _ in range(args.warmup):
         flush.fill_(1.0)

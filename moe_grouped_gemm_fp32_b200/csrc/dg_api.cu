@@ -145,11 +145,20 @@ long long timeout_cycles() {
 
 int g_debug_flags = 0;
 
+// DG_VERBOSE=1 prints each launch's configuration to stderr.
+bool verbose() {
+    static bool v = [] {
+        const char *s = std::getenv("DG_VERBOSE");
+        return s && s[0] == '1';
+    }();
+    return v;
+}
+
 // ------------------------------------------------------------------ launch
 template <int kBN, bool kSwap, int kStages, int kLayout>
 dg_status_t launch(const CUtensorMap &ma, const CUtensorMap &mb, const dg::Params &p, int grid_x,
                    int grid_y, int cluster_x, cudaStream_t stream) {
-    using L = dg::SmemLayout<kBN, kStages>;
+    using L = dg::SmemLayout<kBN, kSwap, kStages>;
     auto kernel = dg::fp8_gemm_kernel<kBN, kSwap, kStages, kLayout>;
     static bool attr_done[kMaxDevices] = {};
     int dev = 0;
@@ -175,6 +184,12 @@ dg_status_t launch(const CUtensorMap &ma, const CUtensorMap &mb, const dg::Param
         attr[0].val.clusterDim.z = 1;
         cfg.numAttrs = 1;
     }
+    if (verbose())
+        std::fprintf(stderr,
+                     "[dg] layout=%d M=%d N=%d K=%d G=%d tile_n=%d swap=%d stages=%d split=%d "
+                     "grid=%dx%d smem=%d\n",
+                     kLayout, p.M, p.N, p.K, p.G, kBN, int(kSwap), kStages, p.split, grid_x,
+                     grid_y, L::kAlloc);
     cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, ma, mb, p);
     if (e != cudaSuccess) return cuda_fail(e, "cudaLaunchKernelEx");
     return DG_SUCCESS;
@@ -184,7 +199,7 @@ dg_status_t launch(const CUtensorMap &ma, const CUtensorMap &mb, const dg::Param
 // (cached per device and cluster size).  0 if the query fails.
 template <int kBN, bool kSwap, int kStages, int kLayout>
 int max_active_clusters(int cluster_x) {
-    using L = dg::SmemLayout<kBN, kStages>;
+    using L = dg::SmemLayout<kBN, kSwap, kStages>;
     auto kernel = dg::fp8_gemm_kernel<kBN, kSwap, kStages, kLayout>;
     static int cache[kMaxDevices][9] = {};
     int dev = 0;

@@ -194,23 +194,28 @@ struct TileMap {
     }
 };
 
-template <int kBN, int kStages>
+template <int kBN, bool kSwap, int kStages>
 struct SmemLayout {
     static constexpr int kXBytes = kTileX * kBlockK;       // 16 KB
     static constexpr int kYBytes = kBN * kBlockK;
     static constexpr int kStageBytes = kXBytes + kYBytes;
     static constexpr int kStagesBytes = kStages * kStageBytes;
-    static constexpr int kBarOffset = kStagesBytes;
+    // Per-stage scale slot: the tile's token-row scales sA[kb][tok0 ...] (one
+    // float per token row), then the weight-block scale(s) sB[wblk][kb].
+    static constexpr int kScaleRows = kSwap ? kBN : kTileX;
+    static constexpr int kSlotFloats = kScaleRows + 4;
+    static constexpr int kSlotBytes = kSlotFloats * 4;
+    static constexpr int kSlotOffset = kStagesBytes;
+    static constexpr int kBarOffset = kSlotOffset + kStages * kSlotBytes;
     static constexpr int kNumBars = 2 * kStages + 2 + 2 + 1;
     static constexpr int kMiscOffset = kBarOffset + kNumBars * 8;     // tmem addr, abort flag
-    static constexpr int kScaleOffset = (kMiscOffset + 16 + 15) / 16 * 16;
-    static constexpr int kScaleBytes = 2 * 128 * 4;
-    static constexpr int kPrefixOffset = kScaleOffset + kScaleBytes;
+    static constexpr int kPrefixOffset = (kMiscOffset + 16 + 15) / 16 * 16;
     static constexpr int kPrefixBytes = (kMaxGroups + 1) * 4;
     static constexpr int kUsed = kPrefixOffset + kPrefixBytes;
     static constexpr int kAlloc = (kUsed + 1024 > kMinSmem) ? kUsed + 1024 : kMinSmem;
     static constexpr int kTmemCols = 2 * kBN < 32 ? 32 : 2 * kBN;
     static_assert(kStageBytes % 1024 == 0, "stage must keep 1024-byte alignment");
+    static_assert(kSlotBytes % 16 == 0, "bulk copies need 16-byte aligned slots");
     static_assert(kStagesBytes >= kTileX * kBN * 4, "split-K receive buffer reuses the stages");
     static_assert(kAlloc <= 227 * 1024, "shared memory budget");
     static_assert((kTmemCols & (kTmemCols - 1)) == 0, "TMEM allocation is a power of two");
@@ -220,14 +225,14 @@ template <int kBN, bool kSwap, int kStages, int kLayout>
 __global__ void __launch_bounds__(kNumThreads, 1)
 fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                 const Params p) {
-    using L = SmemLayout<kBN, kStages>;
+    using L = SmemLayout<kBN, kSwap, kStages>;
     using TM = TileMap<kBN, kSwap, kLayout>;
     static_assert(kBN == 64 || kBN == 128 || kBN == 256, "tile N");
     static_assert(kSwap || kLayout != kMasked, "masked layout runs in swap mode");
     constexpr int kHalf = kBN / 2;               // columns per promotion warpgroup
     constexpr int kChunk = kHalf > 64 ? 16 : 32; // TMEM columns per load (register budget)
     constexpr int kChunks = kHalf / kChunk;
-    constexpr uint32_t kTxBytes = L::kStageBytes;
+    constexpr int kNumSB = (!kSwap && kBN == 256) ? 2 : 1;   // weight blocks per tile
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
@@ -241,7 +246,8 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
     const uint32_t mma_done_bar = bar_base + 8u * (2 * kStages + 4);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kMiscOffset);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kMiscOffset + 4);
-    float *scale_buf = reinterpret_cast<float *>(smem + L::kScaleOffset);
+    const uint32_t slot_base = s_base + L::kSlotOffset;
+    const float *slots = reinterpret_cast<const float *>(smem + L::kSlotOffset);
     int *prefix = reinterpret_cast<int *>(smem + L::kPrefixOffset);
 
     const int warp = threadIdx.x / 32;
@@ -254,7 +260,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
         ptx::prefetch_tmap(&tm_b);
         for (int s = 0; s < kStages; ++s) {
             ptx::mbar_init(full_bar(s), 1);
-            ptx::mbar_init(empty_bar(s), 1);
+            ptx::mbar_init(empty_bar(s), 1 + 8);   // MMA commit + 8 promotion warps (scales read)
         }
         for (int b = 0; b < 2; ++b) {
             ptx::mbar_init(tfull_bar(b), 1);
@@ -325,11 +331,29 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
                         record_status(p.status, kStatusInvalid, kSiteBadGroup);
                     continue;
                 }
+                const float *sfa_g = p.sfa + (kLayout == kMasked ? static_cast<size_t>(tl.g) * p.num_kb * p.ld_sfa : 0);
+                const float *sfb_g = p.sfb + static_cast<size_t>(tl.g) * p.num_nb * p.num_kb;
+                const int wblk0 = tl.n0 / 128;
+                // token-row scales present in memory for this tile (ld_sfa - tok0 is a multiple of 4)
+                const int sa_rows = min(L::kScaleRows, p.ld_sfa - tl.tok0);
+                const uint32_t sa_bytes = static_cast<uint32_t>(sa_rows) * 4u;
                 for (int kb = kb_begin; kb < kb_end; ++kb) {
                     if (!wait(empty_bar(stage), phase ^ 1u, kSiteProducerEmpty)) { ok = false; break; }
                     const uint32_t sx = s_base + stage * L::kStageBytes;
                     const uint32_t sy = sx + L::kXBytes;
-                    ptx::mbar_arrive_expect_tx(full_bar(stage), kTxBytes);
+                    const uint32_t slot = slot_base + stage * L::kSlotBytes;
+#pragma unroll
+                    for (int i = 0; i < kNumSB; ++i) {
+                        const uint32_t dst = slot + (L::kScaleRows + i) * 4u;
+                        if (wblk0 + i < p.num_nb)
+                            ptx::cp_async_4(dst, sfb_g + static_cast<size_t>(wblk0 + i) * p.num_kb + kb);
+                        else
+                            ptx::st_shared_f32(dst, 0.f);
+                    }
+                    ptx::cp_async_arrive(full_bar(stage));
+                    ptx::mbar_arrive_expect_tx(full_bar(stage), L::kStageBytes + sa_bytes);
+                    ptx::bulk_load(slot, sfa_g + static_cast<size_t>(kb) * p.ld_sfa + tl.tok0, sa_bytes,
+                                   full_bar(stage));
                     if (kSwap) {
                         ptx::tma_load_3d(sx, &tm_b, full_bar(stage), kb * kBlockK, tl.n0, tl.g);
                         ptx::tma_load_3d(sy, &tm_a, full_bar(stage), kb * kBlockK, tl.a_row, tl.a_grp);
@@ -407,50 +431,33 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
     const int quarter = warp & 3;                    // TMEM lane quarter this warp may access
     const int half = promo ? (warp - 2) >> 2 : 0;    // column half
     const int lrow = quarter * 32 + lane;            // tile row = TMEM lane
-    const int wg_tid = promo ? ((warp - 2) & 3) * 32 + lane : 0;
     Tile last_tile{0, 0, 0, 0, 0, 0};
     bool have_tile = false;
     if (promo) {
-        int buf = 0;
-        uint32_t tphase = 0;
+        int stage = 0, buf = 0;
+        uint32_t phase = 0, tphase = 0;
         bool ok = true;
         for (int t = t_first; ok && t < num_tiles; t += t_step) {
             Tile tl;
             if (!TM::decode(t, p, prefix, tl)) continue;
 #pragma unroll
             for (int i = 0; i < kHalf; ++i) acc[i] = 0.f;
-            const float *sfa_g = p.sfa + (kLayout == kMasked ? static_cast<size_t>(tl.g) * p.num_kb * p.ld_sfa : 0);
-            const float *sfb_g = p.sfb + static_cast<size_t>(tl.g) * p.num_nb * p.num_kb;
-            // normal mode: this thread's token row and its weight block
-            const int my_tok = tl.tok0 + lrow;
+            const int my_tok = tl.tok0 + lrow;       // normal mode: this thread's token row
             const bool tok_ok = my_tok < tl.tok_end;
-            const int wblk = kSwap ? tl.n0 / 128 : (tl.n0 + half * kHalf) / 128;
-            const bool wblk_ok = wblk < p.num_nb;
-            // swap mode: the column (token) whose scale this thread stages
-            const int col_tok = tl.tok0 + half * kHalf + wg_tid;
-            const bool col_ok = wg_tid < kHalf && col_tok < tl.tok_end;
             for (int kb = kb_begin; kb < kb_end; ++kb) {
-                const float sb = wblk_ok ? __ldg(sfb_g + static_cast<size_t>(wblk) * p.num_kb + kb) : 0.f;
-                float s_row = 0.f, s_col = 0.f;
+                // the stage's scales: visible once its full barrier completed
+                if (!wait(full_bar(stage), phase, kSitePromoFull)) { ok = false; break; }
+                const float *slot = slots + stage * L::kSlotFloats;
+                float s = 0.f, sb = 0.f;
                 if (!kSwap) {
-                    s_row = tok_ok ? __ldg(sfa_g + static_cast<size_t>(kb) * p.ld_sfa + my_tok) : 0.f;
+                    s = slot[lrow] * slot[L::kScaleRows + (kNumSB == 2 ? half : 0)];
+                    __syncwarp();
+                    if (lane == 0) ptx::mbar_arrive(empty_bar(stage));
                 } else {
-                    s_col = col_ok ? __ldg(sfa_g + static_cast<size_t>(kb) * p.ld_sfa + col_tok) : 0.f;
+                    sb = slot[L::kScaleRows];
                 }
-                ok = wait(tfull_bar(buf), tphase, kSitePromoFull);
-                if (kSwap) {
-                    // Stage this K-block's per-column scales (sA * sB) for the warpgroup.
-                    // The first barrier also votes: if any thread of the warpgroup gave
-                    // up, all of them stop together, so no named barrier is left waiting.
-                    ok = !ptx::named_bar_or(1 + half, 128, !ok);
-                    if (ok) {
-                        if (wg_tid < kHalf) scale_buf[half * 128 + wg_tid] = s_col * sb;
-                        ptx::named_bar_sync(1 + half, 128);
-                    }
-                }
-                if (!ok) break;
+                if (!wait(tfull_bar(buf), tphase, kSitePromoFull)) { ok = false; break; }
                 ptx::tc_fence_after();
-                const float s = s_row * sb;
                 const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
                                        static_cast<uint32_t>(buf * kBN + half * kHalf);
 #pragma unroll
@@ -466,20 +473,26 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
                     }
                     float *a = acc + c * kChunk;
                     if (kSwap) {
-                        const float4 *sc = reinterpret_cast<const float4 *>(scale_buf + half * 128 + c * kChunk);
+                        // column (token) scales, broadcast from the slot
+                        const float4 *sc = reinterpret_cast<const float4 *>(slot + half * kHalf + c * kChunk);
 #pragma unroll
                         for (int i = 0; i < kChunk / 4; ++i) {
                             const float4 q4 = sc[i];
-                            a[4 * i + 0] = fmaf(q4.x, v[4 * i + 0], a[4 * i + 0]);
-                            a[4 * i + 1] = fmaf(q4.y, v[4 * i + 1], a[4 * i + 1]);
-                            a[4 * i + 2] = fmaf(q4.z, v[4 * i + 2], a[4 * i + 2]);
-                            a[4 * i + 3] = fmaf(q4.w, v[4 * i + 3], a[4 * i + 3]);
+                            a[4 * i + 0] = fmaf(q4.x * sb, v[4 * i + 0], a[4 * i + 0]);
+                            a[4 * i + 1] = fmaf(q4.y * sb, v[4 * i + 1], a[4 * i + 1]);
+                            a[4 * i + 2] = fmaf(q4.z * sb, v[4 * i + 2], a[4 * i + 2]);
+                            a[4 * i + 3] = fmaf(q4.w * sb, v[4 * i + 3], a[4 * i + 3]);
                         }
                     } else {
 #pragma unroll
                         for (int i = 0; i < kChunk; ++i) a[i] = fmaf(s, v[i], a[i]);
                     }
                 }
+                if (kSwap) {
+                    __syncwarp();
+                    if (lane == 0) ptx::mbar_arrive(empty_bar(stage));
+                }
+                if (++stage == kStages) { stage = 0; phase ^= 1u; }
                 if (++buf == 2) { buf = 0; tphase ^= 1u; }
             }
             if (!ok) break;
