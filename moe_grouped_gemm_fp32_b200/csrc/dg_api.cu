@@ -295,7 +295,7 @@ dg_status_t dg_fp8_gemm_nt(const uint8_t *a, const float *sfa, int ld_sfa, const
                   : bn == 128 ? choose_split<128, dg::kDense>(tiles, p.num_kb, info->num_sms)
                               : choose_split<256, dg::kDense>(tiles, p.num_kb, info->num_sms);
         if ((st = make_map(&mb, b, K, N, 1, 128)) != DG_SUCCESS) return st;
-        if ((st = make_map(&ma, a, K, M, 1, bn)) != DG_SUCCESS) return st;
+        if ((st = make_map(&ma, a, K, M, 1, 32)) != DG_SUCCESS) return st;   // 32-token boxes
         const int gx = p.split > 1 ? p.split : (tiles < info->num_sms ? tiles : info->num_sms);
         const int gy = p.split > 1 ? tiles : 1;
         if (bn == 64) return launch<64, true, 8, dg::kDense>(ma, mb, p, gx, gy, p.split, s);
@@ -352,7 +352,7 @@ dg_status_t dg_m_grouped_fp8_gemm_nt_masked(const uint8_t *a, const float *sfa, 
     const int bn = Mmax <= 64 ? 64 : (Mmax <= 128 ? 128 : 256);
     CUtensorMap ma, mb;
     if ((st = make_map(&mb, b, K, N, G, 128)) != DG_SUCCESS) return st;
-    if ((st = make_map(&ma, a, K, Mmax, G, bn)) != DG_SUCCESS) return st;
+    if ((st = make_map(&ma, a, K, Mmax, G, 32)) != DG_SUCCESS) return st;   // 32-token boxes
     const int grid = info->num_sms;   // the tile count lives on the device
     if (bn == 64) return launch<64, true, 8, dg::kMasked>(ma, mb, p, grid, 1, 1, s);
     if (bn == 128) return launch<128, true, 6, dg::kMasked>(ma, mb, p, grid, 1, 1, s);

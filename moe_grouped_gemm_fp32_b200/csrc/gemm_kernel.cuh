@@ -126,6 +126,7 @@ struct Tile {
     int tok0;    // first token row (within the group's rows)
     int tok_end; // exclusive bound of valid token rows
     int n0;      // first weight row
+    int ntok;    // token rows of this tile that exist: min(rows per tile, tok_end - tok0)
 };
 
 template <int kBN, bool kSwap, int kLayout>
@@ -163,6 +164,7 @@ struct TileMap {
             tl.a_row = tl.tok0;
             tl.tok_end = mm;
             tl.n0 = wb * kWRows;
+            tl.ntok = min(kTokRows, mm - tl.tok0);
             return true;
         }
         const int nt = (p.M + kTokRows - 1) / kTokRows;
@@ -183,6 +185,7 @@ struct TileMap {
         tl.a_grp = 0;
         tl.tok_end = p.M;
         tl.n0 = wb * kWRows;
+        tl.ntok = min(kTokRows, p.M - tl.tok0);
         tl.g = 0;
         if (kLayout == kContiguous) {
             const int g = __ldg(p.m_indices + tl.tok0);
@@ -233,6 +236,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
     constexpr int kChunk = kHalf > 64 ? 16 : 32; // TMEM columns per load (register budget)
     constexpr int kChunks = kHalf / kChunk;
     constexpr int kNumSB = (!kSwap && kBN == 256) ? 2 : 1;   // weight blocks per tile
+    constexpr int kTokBox = 32;                               // swap mode: token rows per TMA box
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
@@ -335,7 +339,11 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
                 const float *sfb_g = p.sfb + static_cast<size_t>(tl.g) * p.num_nb * p.num_kb;
                 const int wblk0 = tl.n0 / 128;
                 // token-row scales present in memory for this tile (ld_sfa - tok0 is a multiple of 4)
-                const int sa_rows = min(L::kScaleRows, p.ld_sfa - tl.tok0);
+                // swap mode fetches only the tile's token rows, in boxes of kTokBox rows
+                const int nload = kSwap ? (tl.ntok + kTokBox - 1) / kTokBox : 1;
+                const uint32_t y_bytes = kSwap ? static_cast<uint32_t>(nload * kTokBox * kBlockK)
+                                               : static_cast<uint32_t>(L::kYBytes);
+                const int sa_rows = min(kSwap ? nload * kTokBox : L::kScaleRows, p.ld_sfa - tl.tok0);
                 const uint32_t sa_bytes = static_cast<uint32_t>(sa_rows) * 4u;
                 for (int kb = kb_begin; kb < kb_end; ++kb) {
                     if (!wait(empty_bar(stage), phase ^ 1u, kSiteProducerEmpty)) { ok = false; break; }
@@ -351,12 +359,14 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
                             ptx::st_shared_f32(dst, 0.f);
                     }
                     ptx::cp_async_arrive(full_bar(stage));
-                    ptx::mbar_arrive_expect_tx(full_bar(stage), L::kStageBytes + sa_bytes);
+                    ptx::mbar_arrive_expect_tx(full_bar(stage), L::kXBytes + y_bytes + sa_bytes);
                     ptx::bulk_load(slot, sfa_g + static_cast<size_t>(kb) * p.ld_sfa + tl.tok0, sa_bytes,
                                    full_bar(stage));
                     if (kSwap) {
                         ptx::tma_load_3d(sx, &tm_b, full_bar(stage), kb * kBlockK, tl.n0, tl.g);
-                        ptx::tma_load_3d(sy, &tm_a, full_bar(stage), kb * kBlockK, tl.a_row, tl.a_grp);
+                        for (int i = 0; i < nload; ++i)
+                            ptx::tma_load_3d(sy + i * kTokBox * kBlockK, &tm_a, full_bar(stage), kb * kBlockK,
+                                             tl.a_row + i * kTokBox, tl.a_grp);
                     } else {
                         ptx::tma_load_3d(sx, &tm_a, full_bar(stage), kb * kBlockK, tl.a_row, tl.a_grp);
                         ptx::tma_load_3d(sy, &tm_b, full_bar(stage), kb * kBlockK, tl.n0, tl.g);
@@ -391,6 +401,8 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
             for (int t = t_first; ok && t < num_tiles; t += t_step) {
                 Tile tl;
                 if (!TM::decode(t, p, prefix, tl)) continue;
+                const uint32_t idesc =
+                    f8_idesc(kSwap ? (tl.ntok + kTokBox - 1) / kTokBox * kTokBox : kBN);
                 for (int kb = kb_begin; kb < kb_end; ++kb) {
                     if (!wait(tempty_bar(buf), tphase ^ 1u, kSiteMmaTmemEmpty)) { ok = false; break; }
                     if (!wait(full_bar(stage), phase, kSiteMmaFull)) { ok = false; break; }
@@ -401,7 +413,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
                     const uint32_t dtm = tmem_base + static_cast<uint32_t>(buf * kBN);
 #pragma unroll
                     for (int k = 0; k < kBlockK / 32; ++k)
-                        ptx::mma_f8f6f4(dtm, dx + 2u * k, dy + 2u * k, f8_idesc(kBN), k > 0 ? 1u : 0u);
+                        ptx::mma_f8f6f4(dtm, dx + 2u * k, dy + 2u * k, idesc, k > 0 ? 1u : 0u);
                     ptx::mma_commit(empty_bar(stage));
                     ptx::mma_commit(tfull_bar(buf));
                     issued_any = true;
@@ -426,13 +438,24 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
 
     // ============================================================ promotion
     // (warps 2..9; warps 0 and 1 skip straight to the split-K barriers)
+    //
+    // Column ownership.  Normal mode: warpgroup h owns the contiguous columns
+    // [h*kHalf, (h+1)*kHalf) (with kBN = 256 that is exactly one 128-row
+    // weight block, so one sB per thread).  Swap mode: columns are tokens and
+    // the tile may hold fewer than kBN of them, so the chunks of kChunk columns
+    // are dealt alternately (chunk 2c+h to warpgroup h) to keep both
+    // warpgroups busy; chunks past the tile's token count are skipped.
     float acc[kHalf];
     const bool promo = warp >= 2;
     const int quarter = warp & 3;                    // TMEM lane quarter this warp may access
-    const int half = promo ? (warp - 2) >> 2 : 0;    // column half
+    const int half = promo ? (warp - 2) >> 2 : 0;    // warpgroup
     const int lrow = quarter * 32 + lane;            // tile row = TMEM lane
-    Tile last_tile{0, 0, 0, 0, 0, 0};
+    auto col_of = [&](int c) {                       // first tile column of local chunk c
+        return kSwap ? (2 * c + half) * kChunk : half * kHalf + c * kChunk;
+    };
+    Tile last_tile{0, 0, 0, 0, 0, 0, 0};
     bool have_tile = false;
+    int last_nvalid = 0;
     if (promo) {
         int stage = 0, buf = 0;
         uint32_t phase = 0, tphase = 0;
@@ -444,6 +467,9 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
             for (int i = 0; i < kHalf; ++i) acc[i] = 0.f;
             const int my_tok = tl.tok0 + lrow;       // normal mode: this thread's token row
             const bool tok_ok = my_tok < tl.tok_end;
+            // chunks of this warpgroup that hold columns of the tile
+            const int ncols = kSwap ? (tl.ntok + kTokBox - 1) / kTokBox * kTokBox : kBN;
+            const int nvalid = kSwap ? (ncols / kChunk - half + 1) / 2 : kChunks;
             for (int kb = kb_begin; kb < kb_end; ++kb) {
                 // the stage's scales: visible once its full barrier completed
                 if (!wait(full_bar(stage), phase, kSitePromoFull)) { ok = false; break; }
@@ -459,33 +485,40 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
                 if (!wait(tfull_bar(buf), tphase, kSitePromoFull)) { ok = false; break; }
                 ptx::tc_fence_after();
                 const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
-                                       static_cast<uint32_t>(buf * kBN + half * kHalf);
+                                       static_cast<uint32_t>(buf * kBN);
+                if (nvalid == 0) {
+                    ptx::tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) ptx::mbar_arrive(tempty_bar(buf));
+                }
 #pragma unroll
                 for (int c = 0; c < kChunks; ++c) {
-                    float v[kChunk];
-                    if constexpr (kChunk == 32) ptx::tmem_ld32(taddr + c * kChunk, v);
-                    else ptx::tmem_ld16(taddr + c * kChunk, v);
-                    ptx::tmem_wait_ld();
-                    if (c == kChunks - 1) {
-                        ptx::tc_fence_before();
-                        __syncwarp();
-                        if (lane == 0) ptx::mbar_arrive(tempty_bar(buf));
-                    }
-                    float *a = acc + c * kChunk;
-                    if (kSwap) {
-                        // column (token) scales, broadcast from the slot
-                        const float4 *sc = reinterpret_cast<const float4 *>(slot + half * kHalf + c * kChunk);
-#pragma unroll
-                        for (int i = 0; i < kChunk / 4; ++i) {
-                            const float4 q4 = sc[i];
-                            a[4 * i + 0] = fmaf(q4.x * sb, v[4 * i + 0], a[4 * i + 0]);
-                            a[4 * i + 1] = fmaf(q4.y * sb, v[4 * i + 1], a[4 * i + 1]);
-                            a[4 * i + 2] = fmaf(q4.z * sb, v[4 * i + 2], a[4 * i + 2]);
-                            a[4 * i + 3] = fmaf(q4.w * sb, v[4 * i + 3], a[4 * i + 3]);
+                    if (c < nvalid) {
+                        float v[kChunk];
+                        if constexpr (kChunk == 32) ptx::tmem_ld32(taddr + col_of(c), v);
+                        else ptx::tmem_ld16(taddr + col_of(c), v);
+                        ptx::tmem_wait_ld();
+                        if (c == nvalid - 1) {
+                            ptx::tc_fence_before();
+                            __syncwarp();
+                            if (lane == 0) ptx::mbar_arrive(tempty_bar(buf));
                         }
-                    } else {
+                        float *a = acc + c * kChunk;
+                        if (kSwap) {
+                            // column (token) scales, broadcast from the slot
+                            const float4 *sc = reinterpret_cast<const float4 *>(slot + col_of(c));
 #pragma unroll
-                        for (int i = 0; i < kChunk; ++i) a[i] = fmaf(s, v[i], a[i]);
+                            for (int i = 0; i < kChunk / 4; ++i) {
+                                const float4 q4 = sc[i];
+                                a[4 * i + 0] = fmaf(q4.x * sb, v[4 * i + 0], a[4 * i + 0]);
+                                a[4 * i + 1] = fmaf(q4.y * sb, v[4 * i + 1], a[4 * i + 1]);
+                                a[4 * i + 2] = fmaf(q4.z * sb, v[4 * i + 2], a[4 * i + 2]);
+                                a[4 * i + 3] = fmaf(q4.w * sb, v[4 * i + 3], a[4 * i + 3]);
+                            }
+                        } else {
+#pragma unroll
+                            for (int i = 0; i < kChunk; ++i) a[i] = fmaf(s, v[i], a[i]);
+                        }
                     }
                 }
                 if (kSwap) {
@@ -497,6 +530,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
             }
             if (!ok) break;
             last_tile = tl;
+            last_nvalid = nvalid;
             have_tile = true;
             if (clustered) break;   // one tile; reduced below
             // ------------------------------------------------ epilogue (direct)
@@ -525,10 +559,16 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
                 const int n = tl.n0 + lrow;
                 if (n < p.N) {
 #pragma unroll
-                    for (int j = 0; j < kHalf; ++j) {
-                        const int m = tl.tok0 + half * kHalf + j;
-                        if (m < tl.tok_end)
-                            p.d[(row_base + m) * static_cast<size_t>(p.N) + n] = __float2bfloat16_rn(acc[j]);
+                    for (int c = 0; c < kChunks; ++c) {
+                        if (c < nvalid) {
+#pragma unroll
+                            for (int i = 0; i < kChunk; ++i) {
+                                const int m = tl.tok0 + col_of(c) + i;
+                                if (m < tl.tok_end)
+                                    p.d[(row_base + m) * static_cast<size_t>(p.N) + n] =
+                                        __float2bfloat16_rn(acc[c * kChunk + i]);
+                            }
+                        }
                     }
                 }
             }
@@ -544,14 +584,21 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
         const int rows_per = kTileX / split;             // split divides 128 (1,2,4,8)
         const uint32_t my_rank = ptx::cluster_rank();
         if (promo && have_tile && !*abort_flag) {
-            // (2) send this thread's row to its owner: slot [src rank][row % rows_per][col]
+            // (2) send this thread's row to its owner: slot [src rank][row % rows_per][column]
             const int owner = lrow / rows_per;
             const uint32_t local = s_base + static_cast<uint32_t>(
-                ((my_rank * rows_per + (lrow % rows_per)) * kBN + half * kHalf) * 4);
+                ((my_rank * rows_per + (lrow % rows_per)) * kBN) * 4);
             const uint32_t remote = ptx::map_cluster(local, static_cast<uint32_t>(owner));
 #pragma unroll
-            for (int j = 0; j < kHalf; j += 4)
-                ptx::st_cluster_v4(remote + j * 4, acc[j], acc[j + 1], acc[j + 2], acc[j + 3]);
+            for (int c = 0; c < kChunks; ++c) {
+                if (c < last_nvalid) {
+#pragma unroll
+                    for (int i = 0; i < kChunk; i += 4)
+                        ptx::st_cluster_v4(remote + (col_of(c) + i) * 4, acc[c * kChunk + i],
+                                           acc[c * kChunk + i + 1], acc[c * kChunk + i + 2],
+                                           acc[c * kChunk + i + 3]);
+                }
+            }
         }
         ptx::cluster_sync_all();
         // (3) each CTA sums its rows over the source ranks in rank order and stores
@@ -560,7 +607,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
             const Tile &tl = last_tile;
             const size_t row_base = kLayout == kMasked ? static_cast<size_t>(tl.g) * p.M : 0;
             const int tid = (warp - 2) * 32 + lane;        // 0..255
-            const int elems = rows_per * kBN;
+            const int elems = rows_per * tl.ntok;
             for (int e = tid; e < elems; e += 256) {
                 const int rr = e % rows_per;               // consecutive threads: consecutive n
                 const int j = e / rows_per;
