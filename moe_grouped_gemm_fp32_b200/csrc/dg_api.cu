@@ -155,11 +155,11 @@ bool verbose() {
 }
 
 // ------------------------------------------------------------------ launch
-template <int kBN, bool kSwap, int kStages, int kLayout>
+template <int kBN, bool kSwap, int kStages, int kLayout, int kCtaGroup = 1>
 dg_status_t launch(const CUtensorMap &ma, const CUtensorMap &mb, const dg::Params &p, int grid_x,
                    int grid_y, int cluster_x, cudaStream_t stream) {
-    using L = dg::SmemLayout<kBN, kSwap, kStages>;
-    auto kernel = dg::fp8_gemm_kernel<kBN, kSwap, kStages, kLayout>;
+    using L = dg::SmemLayout<kBN, kSwap, kStages, kCtaGroup>;
+    auto kernel = dg::fp8_gemm_kernel<kBN, kSwap, kStages, kLayout, kCtaGroup>;
     static bool attr_done[kMaxDevices] = {};
     int dev = 0;
     cudaGetDevice(&dev);
@@ -167,11 +167,25 @@ dg_status_t launch(const CUtensorMap &ma, const CUtensorMap &mb, const dg::Param
         cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              L::kAlloc);
         if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+        if (!kSwap) {
+            // The register rebalancing inside the kernel (setmaxnreg) is sized for
+            // exactly kRegsLaunch registers per thread at launch; with any other
+            // count the promotion warps' request could never be granted.  Refuse.
+            cudaFuncAttributes fa;
+            if ((e = cudaFuncGetAttributes(&fa, kernel)) != cudaSuccess)
+                return cuda_fail(e, "cudaFuncGetAttributes");
+            if (fa.numRegs != dg::kRegsLaunch) {
+                std::snprintf(t_last_cuda_error, sizeof(t_last_cuda_error),
+                              "kernel built with %d registers per thread, expected %d", fa.numRegs,
+                              dg::kRegsLaunch);
+                return DG_ERR_CUDA;
+            }
+        }
         attr_done[dev] = true;
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid_x, grid_y, 1);
-    cfg.blockDim = dim3(dg::kNumThreads, 1, 1);
+    cfg.blockDim = dim3(dg::num_threads(kSwap), 1, 1);
     cfg.dynamicSmemBytes = L::kAlloc;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
@@ -186,10 +200,10 @@ dg_status_t launch(const CUtensorMap &ma, const CUtensorMap &mb, const dg::Param
     }
     if (verbose())
         std::fprintf(stderr,
-                     "[dg] layout=%d M=%d N=%d K=%d G=%d tile_n=%d swap=%d stages=%d split=%d "
-                     "grid=%dx%d smem=%d\n",
-                     kLayout, p.M, p.N, p.K, p.G, kBN, int(kSwap), kStages, p.split, grid_x,
-                     grid_y, L::kAlloc);
+                     "[dg] layout=%d M=%d N=%d K=%d G=%d tile_n=%d swap=%d stages=%d ctas/mma=%d "
+                     "split=%d grid=%dx%d cluster=%d smem=%d\n",
+                     kLayout, p.M, p.N, p.K, p.G, kBN, int(kSwap), kStages, kCtaGroup, p.split, grid_x,
+                     grid_y, cluster_x, L::kAlloc);
     cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, ma, mb, p);
     if (e != cudaSuccess) return cuda_fail(e, "cudaLaunchKernelEx");
     return DG_SUCCESS;
@@ -197,10 +211,10 @@ dg_status_t launch(const CUtensorMap &ma, const CUtensorMap &mb, const dg::Param
 
 // How many clusters of `cluster_x` CTAs of this kernel can be resident at once
 // (cached per device and cluster size).  0 if the query fails.
-template <int kBN, bool kSwap, int kStages, int kLayout>
+template <int kBN, bool kSwap, int kStages, int kLayout, int kCtaGroup = 1>
 int max_active_clusters(int cluster_x) {
-    using L = dg::SmemLayout<kBN, kSwap, kStages>;
-    auto kernel = dg::fp8_gemm_kernel<kBN, kSwap, kStages, kLayout>;
+    using L = dg::SmemLayout<kBN, kSwap, kStages, kCtaGroup>;
+    auto kernel = dg::fp8_gemm_kernel<kBN, kSwap, kStages, kLayout, kCtaGroup>;
     static int cache[kMaxDevices][9] = {};
     int dev = 0;
     cudaGetDevice(&dev);
@@ -213,7 +227,7 @@ int max_active_clusters(int cluster_x) {
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(cluster_x, 1, 1);
-    cfg.blockDim = dim3(dg::kNumThreads, 1, 1);
+    cfg.blockDim = dim3(dg::num_threads(kSwap), 1, 1);
     cfg.dynamicSmemBytes = L::kAlloc;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -302,13 +316,31 @@ dg_status_t dg_fp8_gemm_nt(const uint8_t *a, const float *sfa, int ld_sfa, const
         if (bn == 128) return launch<128, true, 6, dg::kDense>(ma, mb, p, gx, gy, p.split, s);
         return launch<256, true, 4, dg::kDense>(ma, mb, p, gx, gy, p.split, s);
     }
-    const int bn = N <= 128 ? 128 : 256;
-    const int tiles = ((M + 127) / 128) * ((N + bn - 1) / bn);
-    const int grid = tiles < info->num_sms ? tiles : info->num_sms;
+    if (N <= 128) {
+        const int tiles = ((M + 127) / 128) * ((N + 127) / 128);
+        const int grid = tiles < info->num_sms ? tiles : info->num_sms;
+        if ((st = make_map(&ma, a, K, M, 1, 128)) != DG_SUCCESS) return st;
+        if ((st = make_map(&mb, b, K, N, 1, 128)) != DG_SUCCESS) return st;
+        return launch<128, false, 6, dg::kDense>(ma, mb, p, grid, 1, 1, s);
+    }
+    // CTA pairs: 256 x bn tiles with tcgen05.mma.cta_group::2 (DG_PAIR_N
+    // overrides bn for tuning sweeps)
+    static const int forced_bn = [] {
+        const char *e = std::getenv("DG_PAIR_N");
+        return e ? std::atoi(e) : 0;
+    }();
+    const int bn = (forced_bn == 160 || forced_bn == 224 || forced_bn == 256) ? forced_bn : 224;
+    const int pairs_max = bn == 160   ? max_active_clusters<160, false, 7, dg::kDense, 2>(2)
+                          : bn == 224 ? max_active_clusters<224, false, 6, dg::kDense, 2>(2)
+                                      : max_active_clusters<256, false, 6, dg::kDense, 2>(2);
+    if (pairs_max <= 0) return cuda_fail(cudaErrorInvalidConfiguration, "no resident CTA pair");
+    const int tiles = ((M + 255) / 256) * ((N + bn - 1) / bn);
+    const int pairs = tiles < pairs_max ? tiles : pairs_max;
     if ((st = make_map(&ma, a, K, M, 1, 128)) != DG_SUCCESS) return st;
-    if ((st = make_map(&mb, b, K, N, 1, bn)) != DG_SUCCESS) return st;
-    if (bn == 128) return launch<128, false, 6, dg::kDense>(ma, mb, p, grid, 1, 1, s);
-    return launch<256, false, 4, dg::kDense>(ma, mb, p, grid, 1, 1, s);
+    if ((st = make_map(&mb, b, K, N, 1, bn / 2)) != DG_SUCCESS) return st;
+    if (bn == 160) return launch<160, false, 7, dg::kDense, 2>(ma, mb, p, 2 * pairs, 1, 2, s);
+    if (bn == 224) return launch<224, false, 6, dg::kDense, 2>(ma, mb, p, 2 * pairs, 1, 2, s);
+    return launch<256, false, 6, dg::kDense, 2>(ma, mb, p, 2 * pairs, 1, 2, s);
 }
 
 dg_status_t dg_m_grouped_fp8_gemm_nt_contiguous(const uint8_t *a, const float *sfa, int ld_sfa,
@@ -349,14 +381,15 @@ dg_status_t dg_m_grouped_fp8_gemm_nt_masked(const uint8_t *a, const float *sfa, 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     dg::Params p = base_params(sfa, ld_sfa, sfb, d, Mmax, N, K, G, info);
     p.masked_m = masked_m;
-    const int bn = Mmax <= 64 ? 64 : (Mmax <= 128 ? 128 : 256);
+    // at most 128 token columns per tile: all of a thread's columns stay in
+    // registers (larger Mmax takes several token blocks per group)
+    const int bn = Mmax <= 64 ? 64 : 128;
     CUtensorMap ma, mb;
     if ((st = make_map(&mb, b, K, N, G, 128)) != DG_SUCCESS) return st;
     if ((st = make_map(&ma, a, K, Mmax, G, 32)) != DG_SUCCESS) return st;   // 32-token boxes
     const int grid = info->num_sms;   // the tile count lives on the device
     if (bn == 64) return launch<64, true, 8, dg::kMasked>(ma, mb, p, grid, 1, 1, s);
-    if (bn == 128) return launch<128, true, 6, dg::kMasked>(ma, mb, p, grid, 1, 1, s);
-    return launch<256, true, 4, dg::kMasked>(ma, mb, p, grid, 1, 1, s);
+    return launch<128, true, 6, dg::kMasked>(ma, mb, p, grid, 1, 1, s);
 }
 
 int dg_get_m_alignment_for_contiguous_layout(void) { return 128; }

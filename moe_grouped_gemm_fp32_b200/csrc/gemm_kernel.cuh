@@ -4,23 +4,36 @@
 // pages: page 2 "六大核心技术突破" items 1, 4 and 5 -- TMA loads, persistent
 // warp specialisation overlapping data movement, tensor-core MMA and CUDA-core
 // promotion, one block scheduler for dense and grouped GEMMs; page 5 "03" --
-// swapAB on Blackwell for skinny token matrices):
+// swapAB on Blackwell for skinny token matrices; the 2-CTA pair below is the
+// Blackwell counterpart of the pages' TMA multicast of a shared operand):
 //
-//   warp 0      producer: one thread issues TMA tile loads of both operands
-//               for one 128-wide K-block per pipeline stage (128B swizzle).
+//   warp 0      producer: one thread issues, per 128-wide K-block and pipeline
+//               stage, TMA tile loads of both operands (128B swizzle), a bulk
+//               copy of the tile's activation scales and cp.async of the
+//               weight-block scale(s) into the stage's scale slot.
 //   warp 1      TMEM allocator + MMA issuer: one thread issues 4 x
 //               tcgen05.mma.kind::f8f6f4 (K = 32 each) per K-block into a
-//               fresh FP32 partial in TMEM (two partial buffers, ping-pong).
-//   warps 2..9  promotion + epilogue (two warpgroups, each owning half of the
-//               tile's columns): tcgen05.ld the partial, acc += (sA*sB)*P in
-//               FP32 registers, release the partial; after the last K-block
+//               fresh FP32 partial in TMEM (2-4 partial buffers in rotation).
+//   warps 2..9  promotion + epilogue (two warpgroups): read the stage's
+//               scales, tcgen05.ld the partial, acc += (sA*sB)*P in FP32
+//               registers, release the partial; after the last K-block
 //               convert to BF16 and store.
 //
-// Operand roles.  The MMA's "M" side is 128 TMEM lanes; its "N" side is kBN
-// columns.  Normal mode puts 128 token rows of A on lanes and kBN weight rows
-// of B on columns.  Swap-AB mode (small token counts) computes D^T = B * A^T:
-// 128 weight rows on lanes, kBN token rows on columns, so a 64-token decode
-// batch does not waste half of a 128-lane MMA.  Both operands stay K-major.
+// Operand roles.  The MMA's "M" side is 128 TMEM lanes per CTA; its "N" side
+// is kBN columns.  Normal mode puts 128 token rows of A on lanes and kBN
+// weight rows of B on columns.  Swap-AB mode (small token counts) computes
+// D^T = B * A^T: 128 weight rows on lanes, up to kBN token rows on columns, so
+// a 64-token decode batch does not waste half of a 128-lane MMA; only the
+// token rows present are fetched (32-row boxes) and multiplied (MMA N set per
+// tile).  Both operands stay K-major.
+//
+// CTA pairs (kCtaGroup == 2, normal mode): a cluster of 2 CTAs computes one
+// 256 x kBN tile with tcgen05.mma.cta_group::2.  Each CTA stages its own 128
+// token rows and half of the tile's weight rows, so a stage costs each SM
+// 16 KB + kBN/2 x 128 B instead of 16 KB + kBN x 128 B: twice the MMA work
+// per byte held in shared memory and per byte pulled from L2.  The even CTA
+// issues the MMAs; TMA bytes of both CTAs complete on its barrier, and the
+// MMA completions are multicast to both CTAs' barriers.
 //
 // Split-K (swap mode only): a cluster of `split` CTAs shares one output tile,
 // each CTA takes a contiguous range of K-blocks, and the FP32 partial tiles
@@ -44,10 +57,20 @@ namespace dg {
 enum Layout : int { kDense = 0, kContiguous = 1, kMasked = 2 };
 
 constexpr int kBlockK = 128;         // K-block (one 128-byte swizzled row of FP8)
-constexpr int kTileX = 128;          // MMA M (TMEM lanes)
+constexpr int kTileX = 128;          // MMA M per CTA (TMEM lanes)
 constexpr int kMaxGroups = 1024;     // masked layout, group prefix table in smem
-constexpr int kNumThreads = 320;     // 10 warps
+// Swap mode: 10 warps (producer, MMA, 8 promotion).  Normal mode: 12 warps;
+// warps 0-3 (producer, MMA, two idle) hand registers to the two promotion
+// warpgroups (setmaxnreg), which keep 128 accumulators per thread plus a
+// 64-column TMEM batch.
+__host__ __device__ constexpr int num_threads(bool swap) { return swap ? 320 : 384; }
+constexpr int kRegsLaunch = 168;     // normal mode: per-thread registers at launch (65536 / 384)
+constexpr int kRegsIssue = 56;       // producer / MMA warpgroup after rebalancing
+constexpr int kRegsPromo = 224;      // promotion warpgroups after rebalancing
+static_assert(128 * (kRegsLaunch - kRegsIssue) == 256 * (kRegsPromo - kRegsLaunch),
+              "register rebalancing must add up to the launch pool");
 constexpr int kMinSmem = 120 * 1024; // > half an SM: one CTA per SM (TMEM is never contended)
+constexpr int kTokBox = 32;          // swap mode: token rows per TMA box
 
 // status word layout: low 8 bits = dg_status_t code, bits 8..15 = site, bits 16..31 = CTA
 enum StatusCode : unsigned { kStatusInvalid = 1u, kStatusTimeout = 6u };
@@ -84,12 +107,14 @@ struct BoundedWait {
     unsigned *status;
     long long limit;
 
-    // Returns true when the phase completed; false on timeout or abort.
+    // Returns true when the phase completed; false on timeout or abort.  Each
+    // probe may sleep up to ~20 us waiting for the phase, so the deadline and the
+    // abort flag are checked every few microseconds at most.
     __device__ __forceinline__ bool operator()(uint32_t bar, uint32_t parity, unsigned site) const {
         if (ptx::mbar_try_wait(bar, parity)) return true;
         const long long start = clock64();
         while (true) {
-            if (ptx::mbar_try_wait(bar, parity)) return true;
+            if (ptx::mbar_try_wait_sleep(bar, parity, 20000u)) return true;
             if (*abort_flag) return false;
             if (clock64() - start > limit) {
                 record_status(status, kStatusTimeout, site);
@@ -113,10 +138,15 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
     return d;
 }
 
-// Instruction descriptor: D = F32, A = B = E4M3, both K-major, M = 128, N = n.
-__host__ __device__ constexpr uint32_t f8_idesc(int n) {
-    return (1u << 4) | (static_cast<uint32_t>(n >> 3) << 17) |
-           (static_cast<uint32_t>(kTileX >> 4) << 24);
+// Instruction descriptor: D = F32, A = B = E4M3, both K-major, M = m, N = n.
+__host__ __device__ constexpr uint32_t f8_idesc(int m, int n) {
+    return (1u << 4) | (static_cast<uint32_t>(n >> 3) << 17) | (static_cast<uint32_t>(m >> 4) << 24);
+}
+
+// Weight-block scales a tile of bn weight rows starting at a multiple of bn
+// can touch (bn = 224 tiles start at multiples of 32 inside a block).
+__host__ __device__ constexpr int weight_blocks_per_tile(int bn) {
+    return (128 % bn == 0) ? 1 : (bn % 128 == 0 ? bn / 128 : bn / 128 + 2);
 }
 
 struct Tile {
@@ -129,11 +159,11 @@ struct Tile {
     int ntok;    // token rows of this tile that exist: min(rows per tile, tok_end - tok0)
 };
 
-template <int kBN, bool kSwap, int kLayout>
+template <int kBN, bool kSwap, int kLayout, int kCtaGroup>
 struct TileMap {
-    static constexpr int kTokRows = kSwap ? kBN : kTileX;     // token rows per tile
-    static constexpr int kWRows = kSwap ? kTileX : kBN;       // weight rows per tile
-    static constexpr int kRasterM = 16;                       // L2 raster band (token blocks)
+    static constexpr int kTokRows = kSwap ? kBN : kTileX * kCtaGroup;  // token rows per tile
+    static constexpr int kWRows = kSwap ? kTileX : kBN;                // weight rows per tile
+    static constexpr int kRasterM = 16 / kCtaGroup;                    // L2 raster band (token blocks)
 
     // Number of tiles (masked: from the smem prefix table).
     __device__ static int count(const Params &p, const int *prefix) {
@@ -154,10 +184,13 @@ struct TileMap {
                 if (prefix[mid] <= t) lo = mid; else hi = mid - 1;
             }
             const int g = lo, local = t - prefix[g];
-            tb = local / nw;
-            wb = local - tb * nw;
             int mm = p.masked_m[g];
             mm = mm < 0 ? 0 : (mm > p.M ? p.M : mm);
+            // within a group, the token blocks of one weight block are adjacent:
+            // tiles that read the same B rows run at the same time (L2 reuse)
+            const int ntb = (mm + kTokRows - 1) / kTokRows;
+            wb = local / ntb;
+            tb = local - wb * ntb;
             tl.g = g;
             tl.a_grp = g;
             tl.tok0 = tb * kTokRows;
@@ -197,46 +230,61 @@ struct TileMap {
     }
 };
 
-template <int kBN, bool kSwap, int kStages>
+template <int kBN, bool kSwap, int kStages, int kCtaGroup>
 struct SmemLayout {
-    static constexpr int kXBytes = kTileX * kBlockK;       // 16 KB
-    static constexpr int kYBytes = kBN * kBlockK;
+    static constexpr int kYRows = kSwap ? kBN : kBN / kCtaGroup;   // rows of the Y operand per CTA
+    static constexpr int kXBytes = kTileX * kBlockK;               // 16 KB
+    static constexpr int kYBytes = kYRows * kBlockK;
     static constexpr int kStageBytes = kXBytes + kYBytes;
     static constexpr int kStagesBytes = kStages * kStageBytes;
-    // Per-stage scale slot: the tile's token-row scales sA[kb][tok0 ...] (one
+    // Per-stage scale slot: this CTA's token-row scales sA[kb][rows ...] (one
     // float per token row), then the weight-block scale(s) sB[wblk][kb].
     static constexpr int kScaleRows = kSwap ? kBN : kTileX;
-    static constexpr int kSlotFloats = kScaleRows + 4;
+    static constexpr int kNumSB = kSwap ? 1 : weight_blocks_per_tile(kBN);
+    static constexpr int kSlotFloats = kScaleRows + (kNumSB + 3) / 4 * 4;
     static constexpr int kSlotBytes = kSlotFloats * 4;
     static constexpr int kSlotOffset = kStagesBytes;
     static constexpr int kBarOffset = kSlotOffset + kStages * kSlotBytes;
-    static constexpr int kNumBars = 2 * kStages + 2 + 2 + 1;
+    // TMEM partial buffers: as many kBN-column buffers as fit in 512 columns (2..4).
+    // Each K-block's partial lives from its MMA until the promotion warps have
+    // read it; more buffers let the MMAs run further ahead of the promotion.
+    static constexpr int kAccBufs = 512 / kBN >= 4 ? 4 : (512 / kBN >= 3 ? 3 : 2);
+    static constexpr int kNumBars = 2 * kStages + 2 * kAccBufs + 1;
     static constexpr int kMiscOffset = kBarOffset + kNumBars * 8;     // tmem addr, abort flag
     static constexpr int kPrefixOffset = (kMiscOffset + 16 + 15) / 16 * 16;
     static constexpr int kPrefixBytes = (kMaxGroups + 1) * 4;
     static constexpr int kUsed = kPrefixOffset + kPrefixBytes;
     static constexpr int kAlloc = (kUsed + 1024 > kMinSmem) ? kUsed + 1024 : kMinSmem;
-    static constexpr int kTmemCols = 2 * kBN < 32 ? 32 : 2 * kBN;
+    static constexpr int kTmemCols = kAccBufs * kBN <= 32    ? 32
+                                     : kAccBufs * kBN <= 64  ? 64
+                                     : kAccBufs * kBN <= 128 ? 128
+                                     : kAccBufs * kBN <= 256 ? 256 : 512;
+    static_assert(kAccBufs * kBN <= 512, "TMEM holds 512 columns");
+    static constexpr int kRecvStride = kBN + 4;   // split-K receive rows, padded (bank spread)
     static_assert(kStageBytes % 1024 == 0, "stage must keep 1024-byte alignment");
     static_assert(kSlotBytes % 16 == 0, "bulk copies need 16-byte aligned slots");
-    static_assert(kStagesBytes >= kTileX * kBN * 4, "split-K receive buffer reuses the stages");
+    static_assert(!kSwap || kStagesBytes >= kTileX * kRecvStride * 4,
+                  "split-K receive buffer reuses the stages");
     static_assert(kAlloc <= 227 * 1024, "shared memory budget");
-    static_assert((kTmemCols & (kTmemCols - 1)) == 0, "TMEM allocation is a power of two");
 };
 
-template <int kBN, bool kSwap, int kStages, int kLayout>
-__global__ void __launch_bounds__(kNumThreads, 1)
+template <int kBN, bool kSwap, int kStages, int kLayout, int kCtaGroup>
+__global__ void __launch_bounds__(num_threads(kSwap), 1)
 fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                 const Params p) {
-    using L = SmemLayout<kBN, kSwap, kStages>;
-    using TM = TileMap<kBN, kSwap, kLayout>;
-    static_assert(kBN == 64 || kBN == 128 || kBN == 256, "tile N");
+    using L = SmemLayout<kBN, kSwap, kStages, kCtaGroup>;
+    using TM = TileMap<kBN, kSwap, kLayout, kCtaGroup>;
+    static_assert(kBN == 64 || kBN == 128 || kBN == 160 || kBN == 224 || kBN == 256, "tile N");
     static_assert(kSwap || kLayout != kMasked, "masked layout runs in swap mode");
+    static_assert(kCtaGroup == 1 || (kCtaGroup == 2 && !kSwap && kLayout == kDense),
+                  "CTA pairs: dense normal mode");
+    constexpr bool kPair = kCtaGroup == 2;
     constexpr int kHalf = kBN / 2;               // columns per promotion warpgroup
     constexpr int kChunk = kHalf > 64 ? 16 : 32; // TMEM columns per load (register budget)
     constexpr int kChunks = kHalf / kChunk;
-    constexpr int kNumSB = (!kSwap && kBN == 256) ? 2 : 1;   // weight blocks per tile
-    constexpr int kTokBox = 32;                               // swap mode: token rows per TMA box
+    constexpr int kNumSB = L::kNumSB;
+    constexpr int kPromoWarp0 = kSwap ? 2 : 4;    // first promotion warp
+    static_assert(kHalf % kChunk == 0, "chunking");
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
@@ -245,9 +293,10 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
     const uint32_t bar_base = s_base + L::kBarOffset;
     auto full_bar = [&](int s) { return bar_base + 8u * s; };
     auto empty_bar = [&](int s) { return bar_base + 8u * (kStages + s); };
+    constexpr int kAccBufs = L::kAccBufs;
     auto tfull_bar = [&](int b) { return bar_base + 8u * (2 * kStages + b); };
-    auto tempty_bar = [&](int b) { return bar_base + 8u * (2 * kStages + 2 + b); };
-    const uint32_t mma_done_bar = bar_base + 8u * (2 * kStages + 4);
+    auto tempty_bar = [&](int b) { return bar_base + 8u * (2 * kStages + kAccBufs + b); };
+    const uint32_t mma_done_bar = bar_base + 8u * (2 * kStages + 2 * kAccBufs);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kMiscOffset);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kMiscOffset + 4);
     const uint32_t slot_base = s_base + L::kSlotOffset;
@@ -257,6 +306,10 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
     const int warp = threadIdx.x / 32;
     const int lane = threadIdx.x % 32;
     const BoundedWait wait{abort_flag, p.status, p.timeout_cycles};
+    // CTA pair: rank 0 issues the MMAs; its barriers count both CTAs' operand bytes
+    const uint32_t pair_rank = kPair ? (ptx::cluster_rank() & 1u) : 0u;
+    const bool mma_cta = pair_rank == 0;
+    auto leader_addr = [&](uint32_t local) { return kPair ? ptx::map_cluster(local, 0) : local; };
 
     // ------------------------------------------------------------ set-up
     if (threadIdx.x == 0) {
@@ -266,15 +319,15 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
             ptx::mbar_init(full_bar(s), 1);
             ptx::mbar_init(empty_bar(s), 1 + 8);   // MMA commit + 8 promotion warps (scales read)
         }
-        for (int b = 0; b < 2; ++b) {
+        for (int b = 0; b < kAccBufs; ++b) {
             ptx::mbar_init(tfull_bar(b), 1);
-            ptx::mbar_init(tempty_bar(b), 8);
+            ptx::mbar_init(tempty_bar(b), 8 * kCtaGroup);   // every promotion warp of the pair
         }
         ptx::mbar_init(mma_done_bar, 1);
         *abort_flag = 0;
         ptx::fence_mbar_init();
     }
-    if (kLayout == kMasked && warp == 2) {
+    if (kLayout == kMasked && warp == kPromoWarp0) {
         // exclusive prefix of tiles per group: ceil(masked_m[g] / kTokRows) * weight blocks
         const int nw = (p.N + TM::kWRows - 1) / TM::kWRows;
         int carry = 0;
@@ -301,26 +354,40 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
         if (lane == 0) prefix[p.G] = carry;
     }
     if (warp == 1) {
-        ptx::tmem_alloc(ptx::smem_u32(tmem_slot), L::kTmemCols);
-        ptx::tmem_relinquish();
+        if constexpr (kPair) {
+            ptx::tmem_alloc_pair(ptx::smem_u32(tmem_slot), L::kTmemCols);
+            ptx::tmem_relinquish_pair();
+        } else {
+            ptx::tmem_alloc(ptx::smem_u32(tmem_slot), L::kTmemCols);
+            ptx::tmem_relinquish();
+        }
     }
     ptx::tc_fence_before();
     __syncthreads();
+    if constexpr (kPair) ptx::cluster_sync_all();   // the peer's barriers exist before any remote use
     ptx::tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
 
     // tile iteration: persistent (split == 1) or one tile per cluster (split > 1)
-    const bool clustered = p.split > 1;
+    const bool clustered = kSwap && kLayout == kDense && p.split > 1;   // split-K is a dense swap-mode path
     const int num_tiles = clustered ? static_cast<int>(gridDim.y) : TM::count(p, prefix);
-    const int t_first = clustered ? static_cast<int>(blockIdx.y) : static_cast<int>(blockIdx.x);
-    const int t_step = clustered ? num_tiles : static_cast<int>(gridDim.x);
+    const int t_first = clustered ? static_cast<int>(blockIdx.y) : static_cast<int>(blockIdx.x) / kCtaGroup;
+    const int t_step = clustered ? num_tiles : static_cast<int>(gridDim.x) / kCtaGroup;
     int kb_begin = 0, kb_end = p.num_kb;
     if (clustered) {
         const int r = static_cast<int>(ptx::cluster_rank());
         kb_begin = (p.num_kb * r) / p.split;
         kb_end = (p.num_kb * (r + 1)) / p.split;
     }
+    // this CTA's token rows inside a (pair) tile
+    const int my_row0 = kPair ? static_cast<int>(pair_rank) * kTileX : 0;
 
+    // The two role groups below never share code after this point: the
+    // register rebalancing (setmaxnreg) gives each its own budget, which the
+    // compiler can only honour on disjoint paths.  Each group runs its own copy
+    // of the teardown barriers.
+    if (warp < kPromoWarp0) {
+    if constexpr (!kSwap) ptx::regs_dec<kRegsIssue>();
     if (warp == 0) {
         // ======================================================== producer
         if (ptx::elect_one()) {
@@ -338,13 +405,17 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
                 const float *sfa_g = p.sfa + (kLayout == kMasked ? static_cast<size_t>(tl.g) * p.num_kb * p.ld_sfa : 0);
                 const float *sfb_g = p.sfb + static_cast<size_t>(tl.g) * p.num_nb * p.num_kb;
                 const int wblk0 = tl.n0 / 128;
-                // token-row scales present in memory for this tile (ld_sfa - tok0 is a multiple of 4)
                 // swap mode fetches only the tile's token rows, in boxes of kTokBox rows
                 const int nload = kSwap ? (tl.ntok + kTokBox - 1) / kTokBox : 1;
                 const uint32_t y_bytes = kSwap ? static_cast<uint32_t>(nload * kTokBox * kBlockK)
                                                : static_cast<uint32_t>(L::kYBytes);
-                const int sa_rows = min(kSwap ? nload * kTokBox : L::kScaleRows, p.ld_sfa - tl.tok0);
+                // this CTA's token-row scales present in memory (ld_sfa - row0 is a multiple of 4)
+                const int sa_row0 = tl.tok0 + my_row0;
+                const int sa_rows = max(0, min(kSwap ? nload * kTokBox : L::kScaleRows, p.ld_sfa - sa_row0));
                 const uint32_t sa_bytes = static_cast<uint32_t>(sa_rows) * 4u;
+                // operand bytes on this CTA's full barrier (a pair's MMA CTA counts both CTAs')
+                const uint32_t op_bytes = kPair ? (mma_cta ? 2u * (L::kXBytes + y_bytes) : 0u)
+                                                : L::kXBytes + y_bytes;
                 for (int kb = kb_begin; kb < kb_end; ++kb) {
                     if (!wait(empty_bar(stage), phase ^ 1u, kSiteProducerEmpty)) { ok = false; break; }
                     const uint32_t sx = s_base + stage * L::kStageBytes;
@@ -359,14 +430,21 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
                             ptx::st_shared_f32(dst, 0.f);
                     }
                     ptx::cp_async_arrive(full_bar(stage));
-                    ptx::mbar_arrive_expect_tx(full_bar(stage), L::kXBytes + y_bytes + sa_bytes);
-                    ptx::bulk_load(slot, sfa_g + static_cast<size_t>(kb) * p.ld_sfa + tl.tok0, sa_bytes,
-                                   full_bar(stage));
+                    ptx::mbar_arrive_expect_tx(full_bar(stage), op_bytes + sa_bytes);
+                    if (sa_bytes)
+                        ptx::bulk_load(slot, sfa_g + static_cast<size_t>(kb) * p.ld_sfa + sa_row0, sa_bytes,
+                                       full_bar(stage));
                     if (kSwap) {
                         ptx::tma_load_3d(sx, &tm_b, full_bar(stage), kb * kBlockK, tl.n0, tl.g);
                         for (int i = 0; i < nload; ++i)
                             ptx::tma_load_3d(sy + i * kTokBox * kBlockK, &tm_a, full_bar(stage), kb * kBlockK,
                                              tl.a_row + i * kTokBox, tl.a_grp);
+                    } else if (kPair) {
+                        // both CTAs' operand bytes complete on the MMA CTA's barrier
+                        const uint32_t fb = leader_addr(full_bar(stage));
+                        ptx::tma_load_3d_pair(sx, &tm_a, fb, kb * kBlockK, tl.a_row + my_row0, tl.a_grp);
+                        ptx::tma_load_3d_pair(sy, &tm_b, fb, kb * kBlockK,
+                                              tl.n0 + static_cast<int>(pair_rank) * L::kYRows, tl.g);
                     } else {
                         ptx::tma_load_3d(sx, &tm_a, full_bar(stage), kb * kBlockK, tl.a_row, tl.a_grp);
                         ptx::tma_load_3d(sy, &tm_b, full_bar(stage), kb * kBlockK, tl.n0, tl.g);
@@ -376,7 +454,10 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
                 }
             }
             // wind-down: never leave with TMA writes into this CTA's smem in flight
-            // (the last kStages loads sit on distinct stages)
+            // (the last kStages loads sit on distinct stages).  A pair's second CTA
+            // cannot see its operand bytes land on its own barrier; for it the final
+            // cluster barrier, reached only after the MMA CTA consumed every stage or
+            // ran out of time waiting for it, covers them.
             const long long first = issued > kStages ? issued - kStages : 0;
             for (long long i = first; i < issued; ++i) {
                 const int s = static_cast<int>(i % kStages);
@@ -393,7 +474,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
         __syncwarp();
     } else if (warp == 1) {
         // ======================================================== MMA issuer
-        if (ptx::elect_one()) {
+        if (mma_cta && ptx::elect_one()) {
             int stage = 0, buf = 0;
             uint32_t phase = 0, tphase = 0;
             bool issued_any = false;
@@ -401,8 +482,8 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
             for (int t = t_first; ok && t < num_tiles; t += t_step) {
                 Tile tl;
                 if (!TM::decode(t, p, prefix, tl)) continue;
-                const uint32_t idesc =
-                    f8_idesc(kSwap ? (tl.ntok + kTokBox - 1) / kTokBox * kTokBox : kBN);
+                const uint32_t idesc = f8_idesc(kTileX * kCtaGroup,
+                                                kSwap ? (tl.ntok + kTokBox - 1) / kTokBox * kTokBox : kBN);
                 for (int kb = kb_begin; kb < kb_end; ++kb) {
                     if (!wait(tempty_bar(buf), tphase ^ 1u, kSiteMmaTmemEmpty)) { ok = false; break; }
                     if (!wait(full_bar(stage), phase, kSiteMmaFull)) { ok = false; break; }
@@ -411,47 +492,89 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
                     const uint64_t dx = sw128_desc(sx);
                     const uint64_t dy = sw128_desc(sx + L::kXBytes);
                     const uint32_t dtm = tmem_base + static_cast<uint32_t>(buf * kBN);
+                    if constexpr (kPair) {
 #pragma unroll
-                    for (int k = 0; k < kBlockK / 32; ++k)
-                        ptx::mma_f8f6f4(dtm, dx + 2u * k, dy + 2u * k, idesc, k > 0 ? 1u : 0u);
-                    ptx::mma_commit(empty_bar(stage));
-                    ptx::mma_commit(tfull_bar(buf));
+                        for (int k = 0; k < kBlockK / 32; ++k)
+                            ptx::mma_f8f6f4_pair(dtm, dx + 2u * k, dy + 2u * k, idesc, k > 0 ? 1u : 0u);
+                        ptx::mma_commit_pair(empty_bar(stage), 0x3);
+                        ptx::mma_commit_pair(tfull_bar(buf), 0x3);
+                    } else {
+#pragma unroll
+                        for (int k = 0; k < kBlockK / 32; ++k)
+                            ptx::mma_f8f6f4(dtm, dx + 2u * k, dy + 2u * k, idesc, k > 0 ? 1u : 0u);
+                        ptx::mma_commit(empty_bar(stage));
+                        ptx::mma_commit(tfull_bar(buf));
+                    }
                     issued_any = true;
                     if (++stage == kStages) { stage = 0; phase ^= 1u; }
-                    if (++buf == 2) { buf = 0; tphase ^= 1u; }
+                    if (++buf == kAccBufs) { buf = 0; tphase ^= 1u; }
                 }
             }
-            if (issued_any) {
-                // all MMAs of this thread complete before TMEM is released
-                ptx::mma_commit(mma_done_bar);
-                const long long start = clock64();
-                while (!ptx::mbar_try_wait(mma_done_bar, 0)) {
-                    if (clock64() - start > p.timeout_cycles) {
-                        record_status(p.status, kStatusTimeout, kSiteTeardownMma);
-                        break;
-                    }
-                }
-            }
+            // every MMA completes before TMEM is released (a pair tells both CTAs);
+            // the commit is issued even when nothing ran, so the wait below is uniform
+            (void)issued_any;
+            if constexpr (kPair) ptx::mma_commit_pair(mma_done_bar, 0x3);
+            else ptx::mma_commit(mma_done_bar);
         }
         __syncwarp();
     }
 
+    if (clustered) {   // the promotion warps' two split-K cluster barriers
+        __syncwarp();
+        ptx::cluster_sync_all();
+        ptx::cluster_sync_all();
+    }
+    // ------------------------------------------------------------ teardown (issue warps)
+    if (warp == 1 && ptx::elect_one()) {
+        // Every MMA that wrote this CTA's TMEM (or read its smem) has completed.
+        // The MMA CTA committed mma_done after its last MMA (a pair multicasts
+        // it); the wait is bounded.
+        const long long start = clock64();
+        while (!ptx::mbar_try_wait(mma_done_bar, 0)) {
+            if (clock64() - start > p.timeout_cycles) {
+                record_status(p.status, kStatusTimeout, kSiteTeardownMma);
+                break;
+            }
+        }
+    }
+    __syncwarp();
+    ptx::tc_fence_before();
+    __syncthreads();
+    if constexpr (kPair) ptx::cluster_sync_all();   // no CTA leaves while its peer may touch its smem
+    if (warp == 1) {
+        ptx::tc_fence_after();
+        if constexpr (kPair) ptx::tmem_dealloc_pair(tmem_base, L::kTmemCols);
+        else ptx::tmem_dealloc(tmem_base, L::kTmemCols);
+    }
+    } else {
+    if constexpr (!kSwap) ptx::regs_inc<kRegsPromo>();
     // ============================================================ promotion
-    // (warps 2..9; warps 0 and 1 skip straight to the split-K barriers)
+    // (warps kPromoWarp0 and up)
     //
     // Column ownership.  Normal mode: warpgroup h owns the contiguous columns
-    // [h*kHalf, (h+1)*kHalf) (with kBN = 256 that is exactly one 128-row
-    // weight block, so one sB per thread).  Swap mode: columns are tokens and
-    // the tile may hold fewer than kBN of them, so the chunks of kChunk columns
+    // [h*kHalf, (h+1)*kHalf); each chunk of kChunk columns lies inside one
+    // 128-row weight block, whose scale the chunk uses.  Swap mode: columns
+    // are tokens and the tile may hold fewer than kBN of them, so the chunks
     // are dealt alternately (chunk 2c+h to warpgroup h) to keep both
     // warpgroups busy; chunks past the tile's token count are skipped.
     float acc[kHalf];
-    const bool promo = warp >= 2;
+    const bool promo = warp >= kPromoWarp0;
     const int quarter = warp & 3;                    // TMEM lane quarter this warp may access
-    const int half = promo ? (warp - 2) >> 2 : 0;    // warpgroup
+    const int half = promo ? (warp - kPromoWarp0) >> 2 : 0;    // warpgroup
     const int lrow = quarter * 32 + lane;            // tile row = TMEM lane
     auto col_of = [&](int c) {                       // first tile column of local chunk c
         return kSwap ? (2 * c + half) * kChunk : half * kHalf + c * kChunk;
+    };
+    // the partial buffers are released on the MMA CTA's barrier (remote for a pair's second CTA)
+    const bool remote_release = kPair && !mma_cta;
+    const uint32_t tempty_target0 = remote_release ? leader_addr(tempty_bar(0)) : tempty_bar(0);
+    auto release_tmem = [&](uint32_t target) {
+        ptx::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+            if (remote_release) ptx::mbar_arrive_remote(target);
+            else ptx::mbar_arrive(target);
+        }
     };
     Tile last_tile{0, 0, 0, 0, 0, 0, 0};
     bool have_tile = false;
@@ -465,18 +588,22 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
             if (!TM::decode(t, p, prefix, tl)) continue;
 #pragma unroll
             for (int i = 0; i < kHalf; ++i) acc[i] = 0.f;
-            const int my_tok = tl.tok0 + lrow;       // normal mode: this thread's token row
+            const int my_tok = tl.tok0 + my_row0 + lrow;   // normal mode: this thread's token row
             const bool tok_ok = my_tok < tl.tok_end;
             // chunks of this warpgroup that hold columns of the tile
             const int ncols = kSwap ? (tl.ntok + kTokBox - 1) / kTokBox * kTokBox : kBN;
             const int nvalid = kSwap ? (ncols / kChunk - half + 1) / 2 : kChunks;
+            const int wblk0 = tl.n0 / 128;
             for (int kb = kb_begin; kb < kb_end; ++kb) {
                 // the stage's scales: visible once its full barrier completed
                 if (!wait(full_bar(stage), phase, kSitePromoFull)) { ok = false; break; }
                 const float *slot = slots + stage * L::kSlotFloats;
-                float s = 0.f, sb = 0.f;
+                float sa_row = 0.f, sb = 0.f;
+                float sbv[kNumSB];
                 if (!kSwap) {
-                    s = slot[lrow] * slot[L::kScaleRows + (kNumSB == 2 ? half : 0)];
+                    sa_row = slot[lrow];
+#pragma unroll
+                    for (int i = 0; i < kNumSB; ++i) sbv[i] = slot[L::kScaleRows + i];
                     __syncwarp();
                     if (lane == 0) ptx::mbar_arrive(empty_bar(stage));
                 } else {
@@ -486,38 +613,105 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
                 ptx::tc_fence_after();
                 const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
                                        static_cast<uint32_t>(buf * kBN);
-                if (nvalid == 0) {
-                    ptx::tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) ptx::mbar_arrive(tempty_bar(buf));
+                const uint32_t tempty_target = tempty_target0 + 8u * buf;
+                if constexpr (!kSwap && kHalf <= 96) {
+                    // Normal mode, narrow tiles: all kHalf columns of the warpgroup are
+                    // loaded before one wait and the partial buffer is released at once,
+                    // before the FMAs, so the MMA can reuse it as early as possible.
+                    float v[kHalf];
+                    const uint32_t ta = taddr + static_cast<uint32_t>(half * kHalf);
+#pragma unroll
+                    for (int o = 0; o + 32 <= kHalf; o += 32) ptx::tmem_ld32p(ta + o, v + o);
+                    if constexpr (kHalf % 32 >= 16) ptx::tmem_ld16p(ta + kHalf / 32 * 32, v + kHalf / 32 * 32);
+                    if constexpr (kHalf % 16 == 8) ptx::tmem_ld8p(ta + kHalf - 8, v + kHalf - 8);
+                    ptx::tmem_wait_ld();
+                    release_tmem(tempty_target);
+                    float sblk[kNumSB];
+#pragma unroll
+                    for (int i = 0; i < kNumSB; ++i) sblk[i] = sa_row * sbv[i];
+#pragma unroll
+                    for (int q = 0; q < kHalf / 8; ++q) {
+                        const int col = half * kHalf + q * 8;
+                        const int blk = (tl.n0 + col) / 128 - wblk0;
+                        float sc = sblk[0];
+#pragma unroll
+                        for (int i = 1; i < kNumSB; ++i) sc = blk == i ? sblk[i] : sc;
+#pragma unroll
+                        for (int i = 0; i < 8; i += 2)
+                            ptx::ffma2(acc[q * 8 + i], acc[q * 8 + i + 1], sc, v[q * 8 + i], v[q * 8 + i + 1]);
+                    }
+                    if (++stage == kStages) { stage = 0; phase ^= 1u; }
+                    if (++buf == kAccBufs) { buf = 0; tphase ^= 1u; }
+                    continue;
+                } else if constexpr (!kSwap) {
+                    // Normal mode: this warpgroup's kHalf columns in rounds of up to 32;
+                    // each round loads its columns before one wait (the compiler may
+                    // hoist the next round's load above this round's FMAs).  Every
+                    // 8-column group lies inside one 128-row weight block (scale sblk[]).
+                    constexpr int kRounds = (kHalf + 31) / 32;
+                    float sblk[kNumSB];
+#pragma unroll
+                    for (int i = 0; i < kNumSB; ++i) sblk[i] = sa_row * sbv[i];
+#pragma unroll
+                    for (int r = 0; r < kRounds; ++r) {
+                        constexpr int kFull = 32;
+                        const int ncol = (r + 1) * 32 <= kHalf ? kFull : kHalf - r * 32;   // 32 or 16
+                        float v[32];
+                        const uint32_t ta = taddr + static_cast<uint32_t>(half * kHalf + r * 32);
+                        if (ncol == 32) ptx::tmem_ld32p(ta, v);
+                        else ptx::tmem_ld16p(ta, v);
+                        ptx::tmem_wait_ld();
+                        if (r == kRounds - 1) release_tmem(tempty_target);
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            if (q * 8 < ncol) {
+                                const int col = half * kHalf + r * 32 + q * 8;
+                                const int blk = (tl.n0 + col) / 128 - wblk0;
+                                float sc = sblk[0];
+#pragma unroll
+                                for (int i = 1; i < kNumSB; ++i) sc = blk == i ? sblk[i] : sc;
+                                float *a = acc + r * 32 + q * 8;
+#pragma unroll
+                                for (int i = 0; i < 8; i += 2)
+                                    ptx::ffma2(a[i], a[i + 1], sc, v[q * 8 + i], v[q * 8 + i + 1]);
+                            }
+                        }
+                    }
+                    if (++stage == kStages) { stage = 0; phase ^= 1u; }
+                    if (++buf == kAccBufs) { buf = 0; tphase ^= 1u; }
+                    continue;
                 }
+                // Swap mode.  Batched: every chunk of the thread is loaded before one
+                // wait, so the TMEM read latency is paid once per K-block.
+                constexpr bool kBatch = kHalf <= 64 && kChunk == 32;
+                float vb[kBatch ? kHalf : 1];
+                if constexpr (kBatch) {
+#pragma unroll
+                    for (int c = 0; c < kChunks; ++c)
+                        if (c < nvalid) ptx::tmem_ld32p(taddr + col_of(c), vb + c * kChunk);
+                    ptx::tmem_wait_ld();
+                    if (nvalid > 0) release_tmem(tempty_target);
+                }
+                if (nvalid == 0) release_tmem(tempty_target);
 #pragma unroll
                 for (int c = 0; c < kChunks; ++c) {
                     if (c < nvalid) {
-                        float v[kChunk];
-                        if constexpr (kChunk == 32) ptx::tmem_ld32(taddr + col_of(c), v);
-                        else ptx::tmem_ld16(taddr + col_of(c), v);
-                        ptx::tmem_wait_ld();
-                        if (c == nvalid - 1) {
-                            ptx::tc_fence_before();
-                            __syncwarp();
-                            if (lane == 0) ptx::mbar_arrive(tempty_bar(buf));
+                        float vs[kBatch ? 1 : kChunk];
+                        float *v = kBatch ? vb + c * kChunk : vs;
+                        if constexpr (!kBatch) {
+                            if constexpr (kChunk == 32) ptx::tmem_ld32p(taddr + col_of(c), v);
+                            else ptx::tmem_ld16(taddr + col_of(c), vs);
+                            ptx::tmem_wait_ld();
+                            if (c == nvalid - 1) release_tmem(tempty_target);
                         }
                         float *a = acc + c * kChunk;
-                        if (kSwap) {
-                            // column (token) scales, broadcast from the slot
-                            const float4 *sc = reinterpret_cast<const float4 *>(slot + col_of(c));
+                        // column (token) scales, broadcast from the slot
+                        const float4 *sc = reinterpret_cast<const float4 *>(slot + col_of(c));
 #pragma unroll
-                            for (int i = 0; i < kChunk / 4; ++i) {
-                                const float4 q4 = sc[i];
-                                a[4 * i + 0] = fmaf(q4.x * sb, v[4 * i + 0], a[4 * i + 0]);
-                                a[4 * i + 1] = fmaf(q4.y * sb, v[4 * i + 1], a[4 * i + 1]);
-                                a[4 * i + 2] = fmaf(q4.z * sb, v[4 * i + 2], a[4 * i + 2]);
-                                a[4 * i + 3] = fmaf(q4.w * sb, v[4 * i + 3], a[4 * i + 3]);
-                            }
-                        } else {
-#pragma unroll
-                            for (int i = 0; i < kChunk; ++i) a[i] = fmaf(s, v[i], a[i]);
+                        for (int i = 0; i < kChunk / 4; ++i) {
+                            const float4 q4 = sc[i];
+                            ptx::ffma2s(a[4 * i + 0], a[4 * i + 1], q4.x * sb, q4.y * sb, v[4 * i + 0], v[4 * i + 1]);
+                            ptx::ffma2s(a[4 * i + 2], a[4 * i + 3], q4.z * sb, q4.w * sb, v[4 * i + 2], v[4 * i + 3]);
                         }
                     }
                 }
@@ -526,7 +720,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
                     if (lane == 0) ptx::mbar_arrive(empty_bar(stage));
                 }
                 if (++stage == kStages) { stage = 0; phase ^= 1u; }
-                if (++buf == 2) { buf = 0; tphase ^= 1u; }
+                if (++buf == kAccBufs) { buf = 0; tphase ^= 1u; }
             }
             if (!ok) break;
             last_tile = tl;
@@ -587,7 +781,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
             // (2) send this thread's row to its owner: slot [src rank][row % rows_per][column]
             const int owner = lrow / rows_per;
             const uint32_t local = s_base + static_cast<uint32_t>(
-                ((my_rank * rows_per + (lrow % rows_per)) * kBN) * 4);
+                ((my_rank * rows_per + (lrow % rows_per)) * L::kRecvStride) * 4);
             const uint32_t remote = ptx::map_cluster(local, static_cast<uint32_t>(owner));
 #pragma unroll
             for (int c = 0; c < kChunks; ++c) {
@@ -601,32 +795,43 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
             }
         }
         ptx::cluster_sync_all();
-        // (3) each CTA sums its rows over the source ranks in rank order and stores
+        // (3) each CTA sums its rows over the source ranks in rank order and stores.
+        // Thread -> (row rr, 4 columns j4): consecutive threads take consecutive rows,
+        // so a quarter-warp's 16-byte reads hit distinct banks (padded row stride)
+        // and a warp's BF16 stores of one column are contiguous in D.
         if (promo && have_tile) {
-            const float *recv = reinterpret_cast<const float *>(smem);
+            const float4 *recv = reinterpret_cast<const float4 *>(smem);
             const Tile &tl = last_tile;
             const size_t row_base = kLayout == kMasked ? static_cast<size_t>(tl.g) * p.M : 0;
-            const int tid = (warp - 2) * 32 + lane;        // 0..255
-            const int elems = rows_per * tl.ntok;
+            const int tid = (warp - kPromoWarp0) * 32 + lane;        // 0..255
+            const int groups = (tl.ntok + 3) / 4;
+            const int elems = rows_per * groups;
+            const int n = tl.n0 + static_cast<int>(my_rank) * rows_per;
             for (int e = tid; e < elems; e += 256) {
-                const int rr = e % rows_per;               // consecutive threads: consecutive n
-                const int j = e / rows_per;
-                float sum = 0.f;
-                for (int src = 0; src < split; ++src) sum += recv[(src * rows_per + rr) * kBN + j];
-                const int n = tl.n0 + static_cast<int>(my_rank) * rows_per + rr;
-                const int m = tl.tok0 + j;
-                if (n < p.N && m < tl.tok_end)
-                    p.d[(row_base + m) * static_cast<size_t>(p.N) + n] = __float2bfloat16_rn(sum);
+                const int rr = e % rows_per;
+                const int j4 = e / rows_per;
+                float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
+                for (int src = 0; src < split; ++src) {
+                    const float4 v = recv[((src * rows_per + rr) * L::kRecvStride) / 4 + j4];
+                    sum.x += v.x; sum.y += v.y; sum.z += v.z; sum.w += v.w;
+                }
+                const float vals[4] = {sum.x, sum.y, sum.z, sum.w};
+                if (n + rr < p.N) {
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const int m = tl.tok0 + 4 * j4 + q;
+                        if (m < tl.tok_end)
+                            p.d[(row_base + m) * static_cast<size_t>(p.N) + n + rr] = __float2bfloat16_rn(vals[q]);
+                    }
+                }
             }
         }
     }
 
-    // ============================================================ teardown
+    // ------------------------------------------------------------ teardown (promotion warps)
     ptx::tc_fence_before();
     __syncthreads();
-    if (warp == 1) {
-        ptx::tc_fence_after();
-        ptx::tmem_dealloc(tmem_base, L::kTmemCols);
+    if constexpr (kPair) ptx::cluster_sync_all();
     }
 }
 
