@@ -381,15 +381,30 @@ dg_status_t dg_m_grouped_fp8_gemm_nt_masked(const uint8_t *a, const float *sfa, 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     dg::Params p = base_params(sfa, ld_sfa, sfb, d, Mmax, N, K, G, info);
     p.masked_m = masked_m;
-    // at most 128 token columns per tile: all of a thread's columns stay in
-    // registers (larger Mmax takes several token blocks per group)
-    const int bn = Mmax <= 64 ? 64 : 128;
     CUtensorMap ma, mb;
-    if ((st = make_map(&mb, b, K, N, G, 128)) != DG_SUCCESS) return st;
-    if ((st = make_map(&ma, a, K, Mmax, G, 32)) != DG_SUCCESS) return st;   // 32-token boxes
     const int grid = info->num_sms;   // the tile count lives on the device
-    if (bn == 64) return launch<64, true, 8, dg::kMasked>(ma, mb, p, grid, 1, 1, s);
-    return launch<128, true, 6, dg::kMasked>(ma, mb, p, grid, 1, 1, s);
+    static const bool force_swap = [] {
+        const char *e = std::getenv("DG_MASKED_SWAP");
+        return e && e[0] == '1';
+    }();
+    if (force_swap) {
+        // swap-AB tiles: 128 weight rows x up to 128 tokens (DG_MASKED_SWAP=1, comparisons)
+        const int bn = Mmax <= 64 ? 64 : 128;
+        if ((st = make_map(&mb, b, K, N, G, 128)) != DG_SUCCESS) return st;
+        if ((st = make_map(&ma, a, K, Mmax, G, 32)) != DG_SUCCESS) return st;   // 32-token boxes
+        if (bn == 64) return launch<64, true, 8, dg::kMasked>(ma, mb, p, grid, 1, 1, s);
+        return launch<128, true, 6, dg::kMasked>(ma, mb, p, grid, 1, 1, s);
+    }
+    // Normal mode: 128 token rows on the TMEM lanes, so each promotion thread's
+    // token scale is one register and the weight scale is uniform per 128
+    // columns (one FMA per element, no per-column scale traffic).  Groups with
+    // fewer than 128 valid rows leave the other lanes idle; the weight stream,
+    // which bounds this layout, is read once per token block.
+    const int bn = N <= 128 ? 128 : 256;
+    if ((st = make_map(&ma, a, K, Mmax, G, 128)) != DG_SUCCESS) return st;
+    if ((st = make_map(&mb, b, K, N, G, bn)) != DG_SUCCESS) return st;
+    if (bn == 128) return launch<128, false, 6, dg::kMasked>(ma, mb, p, grid, 1, 1, s);
+    return launch<256, false, 4, dg::kMasked>(ma, mb, p, grid, 1, 1, s);
 }
 
 int dg_get_m_alignment_for_contiguous_layout(void) { return 128; }

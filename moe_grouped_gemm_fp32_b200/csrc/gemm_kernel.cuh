@@ -59,11 +59,12 @@ enum Layout : int { kDense = 0, kContiguous = 1, kMasked = 2 };
 constexpr int kBlockK = 128;         // K-block (one 128-byte swizzled row of FP8)
 constexpr int kTileX = 128;          // MMA M per CTA (TMEM lanes)
 constexpr int kMaxGroups = 1024;     // masked layout, group prefix table in smem
-// Swap mode: 10 warps (producer, MMA, 8 promotion).  Normal mode: 12 warps;
-// warps 0-3 (producer, MMA, two idle) hand registers to the two promotion
-// warpgroups (setmaxnreg), which keep 128 accumulators per thread plus a
-// 64-column TMEM batch.
-__host__ __device__ constexpr int num_threads(bool swap) { return swap ? 320 : 384; }
+// Swap mode: 11 warps (producer, MMA, 8 promotion, scale preparation).
+// Normal mode: 12 warps; warps 0-3 (producer, MMA, two idle) hand registers
+// to the two promotion warpgroups (setmaxnreg), which keep up to 128
+// accumulators per thread plus a TMEM batch.
+__host__ __device__ constexpr int num_threads(bool swap) { return swap ? 352 : 384; }
+constexpr int kPrepWarp = 10;        // swap mode: multiplies token scales by the weight scale
 constexpr int kRegsLaunch = 168;     // normal mode: per-thread registers at launch (65536 / 384)
 constexpr int kRegsIssue = 56;       // producer / MMA warpgroup after rebalancing
 constexpr int kRegsPromo = 224;      // promotion warpgroups after rebalancing
@@ -243,13 +244,16 @@ struct SmemLayout {
     static constexpr int kNumSB = kSwap ? 1 : weight_blocks_per_tile(kBN);
     static constexpr int kSlotFloats = kScaleRows + (kNumSB + 3) / 4 * 4;
     static constexpr int kSlotBytes = kSlotFloats * 4;
+    // Swap mode keeps the scale slots in a ring of their own, deeper than the
+    // operand stages, so an operand stage is free as soon as its MMAs ran.
+    static constexpr int kSlots = kSwap ? 16 : kStages;
     static constexpr int kSlotOffset = kStagesBytes;
-    static constexpr int kBarOffset = kSlotOffset + kStages * kSlotBytes;
+    static constexpr int kBarOffset = kSlotOffset + kSlots * kSlotBytes;
     // TMEM partial buffers: as many kBN-column buffers as fit in 512 columns (2..4).
     // Each K-block's partial lives from its MMA until the promotion warps have
     // read it; more buffers let the MMAs run further ahead of the promotion.
     static constexpr int kAccBufs = 512 / kBN >= 4 ? 4 : (512 / kBN >= 3 ? 3 : 2);
-    static constexpr int kNumBars = 2 * kStages + 2 * kAccBufs + 1;
+    static constexpr int kNumBars = 2 * kStages + 2 * kAccBufs + 1 + (kSwap ? 3 * kSlots : 0);
     static constexpr int kMiscOffset = kBarOffset + kNumBars * 8;     // tmem addr, abort flag
     static constexpr int kPrefixOffset = (kMiscOffset + 16 + 15) / 16 * 16;
     static constexpr int kPrefixBytes = (kMaxGroups + 1) * 4;
@@ -275,7 +279,6 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
     using L = SmemLayout<kBN, kSwap, kStages, kCtaGroup>;
     using TM = TileMap<kBN, kSwap, kLayout, kCtaGroup>;
     static_assert(kBN == 64 || kBN == 128 || kBN == 160 || kBN == 224 || kBN == 256, "tile N");
-    static_assert(kSwap || kLayout != kMasked, "masked layout runs in swap mode");
     static_assert(kCtaGroup == 1 || (kCtaGroup == 2 && !kSwap && kLayout == kDense),
                   "CTA pairs: dense normal mode");
     constexpr bool kPair = kCtaGroup == 2;
@@ -297,10 +300,16 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
     auto tfull_bar = [&](int b) { return bar_base + 8u * (2 * kStages + b); };
     auto tempty_bar = [&](int b) { return bar_base + 8u * (2 * kStages + kAccBufs + b); };
     const uint32_t mma_done_bar = bar_base + 8u * (2 * kStages + 2 * kAccBufs);
+    // swap mode scale ring: producer copies -> sfull, scale-prep warp -> sready,
+    // promotion warps done -> sempty
+    constexpr int kSlots = L::kSlots;
+    auto sfull_bar = [&](int i) { return bar_base + 8u * (2 * kStages + 2 * kAccBufs + 1 + i); };
+    auto sready_bar = [&](int i) { return bar_base + 8u * (2 * kStages + 2 * kAccBufs + 1 + kSlots + i); };
+    auto sempty_bar = [&](int i) { return bar_base + 8u * (2 * kStages + 2 * kAccBufs + 1 + 2 * kSlots + i); };
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kMiscOffset);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kMiscOffset + 4);
     const uint32_t slot_base = s_base + L::kSlotOffset;
-    const float *slots = reinterpret_cast<const float *>(smem + L::kSlotOffset);
+    float *slots = reinterpret_cast<float *>(smem + L::kSlotOffset);
     int *prefix = reinterpret_cast<int *>(smem + L::kPrefixOffset);
 
     const int warp = threadIdx.x / 32;
@@ -317,7 +326,15 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
         ptx::prefetch_tmap(&tm_b);
         for (int s = 0; s < kStages; ++s) {
             ptx::mbar_init(full_bar(s), 1);
-            ptx::mbar_init(empty_bar(s), 1 + 8);   // MMA commit + 8 promotion warps (scales read)
+            // MMA commit (+ 8 promotion warps that read the stage's scales, normal mode)
+            ptx::mbar_init(empty_bar(s), kSwap ? 1 : 1 + 8);
+        }
+        if constexpr (kSwap) {
+            for (int i = 0; i < kSlots; ++i) {
+                ptx::mbar_init(sfull_bar(i), 1);
+                ptx::mbar_init(sready_bar(i), 32);
+                ptx::mbar_init(sempty_bar(i), 8);
+            }
         }
         for (int b = 0; b < kAccBufs; ++b) {
             ptx::mbar_init(tfull_bar(b), 1);
@@ -391,8 +408,8 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
     if (warp == 0) {
         // ======================================================== producer
         if (ptx::elect_one()) {
-            int stage = 0;
-            uint32_t phase = 0;
+            int stage = 0, sslot = 0;
+            uint32_t phase = 0, sphase = 0;
             long long issued = 0;
             bool ok = (p.debug_flags & kDebugProducerIdle) == 0;
             for (int t = t_first; ok && t < num_tiles; t += t_step) {
@@ -418,9 +435,11 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
                                                 : L::kXBytes + y_bytes;
                 for (int kb = kb_begin; kb < kb_end; ++kb) {
                     if (!wait(empty_bar(stage), phase ^ 1u, kSiteProducerEmpty)) { ok = false; break; }
+                    if (kSwap && !wait(sempty_bar(sslot), sphase ^ 1u, kSiteProducerEmpty)) { ok = false; break; }
                     const uint32_t sx = s_base + stage * L::kStageBytes;
                     const uint32_t sy = sx + L::kXBytes;
-                    const uint32_t slot = slot_base + stage * L::kSlotBytes;
+                    const uint32_t slot = slot_base + (kSwap ? sslot : stage) * L::kSlotBytes;
+                    const uint32_t scale_bar = kSwap ? sfull_bar(sslot) : full_bar(stage);
 #pragma unroll
                     for (int i = 0; i < kNumSB; ++i) {
                         const uint32_t dst = slot + (L::kScaleRows + i) * 4u;
@@ -429,11 +448,16 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
                         else
                             ptx::st_shared_f32(dst, 0.f);
                     }
-                    ptx::cp_async_arrive(full_bar(stage));
-                    ptx::mbar_arrive_expect_tx(full_bar(stage), op_bytes + sa_bytes);
+                    ptx::cp_async_arrive(scale_bar);
+                    if (kSwap) {
+                        ptx::mbar_arrive_expect_tx(scale_bar, sa_bytes);
+                        ptx::mbar_arrive_expect_tx(full_bar(stage), op_bytes);
+                    } else {
+                        ptx::mbar_arrive_expect_tx(full_bar(stage), op_bytes + sa_bytes);
+                    }
                     if (sa_bytes)
                         ptx::bulk_load(slot, sfa_g + static_cast<size_t>(kb) * p.ld_sfa + sa_row0, sa_bytes,
-                                       full_bar(stage));
+                                       scale_bar);
                     if (kSwap) {
                         ptx::tma_load_3d(sx, &tm_b, full_bar(stage), kb * kBlockK, tl.n0, tl.g);
                         for (int i = 0; i < nload; ++i)
@@ -451,6 +475,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
                     }
                     ++issued;
                     if (++stage == kStages) { stage = 0; phase ^= 1u; }
+                    if (kSwap && ++sslot == kSlots) { sslot = 0; sphase ^= 1u; }
                 }
             }
             // wind-down: never leave with TMA writes into this CTA's smem in flight
@@ -458,18 +483,22 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
             // cannot see its operand bytes land on its own barrier; for it the final
             // cluster barrier, reached only after the MMA CTA consumed every stage or
             // ran out of time waiting for it, covers them.
-            const long long first = issued > kStages ? issued - kStages : 0;
-            for (long long i = first; i < issued; ++i) {
-                const int s = static_cast<int>(i % kStages);
-                const uint32_t par = static_cast<uint32_t>((i / kStages) & 1);
-                const long long start = clock64();
-                while (!ptx::mbar_try_wait(full_bar(s), par)) {
-                    if (clock64() - start > p.timeout_cycles) {
-                        record_status(p.status, kStatusTimeout, kSiteTeardownLoads);
-                        break;
+            auto drain = [&](long long depth, auto bar_of) {
+                const long long first = issued > depth ? issued - depth : 0;
+                for (long long i = first; i < issued; ++i) {
+                    const uint32_t bar = bar_of(static_cast<int>(i % depth));
+                    const uint32_t par = static_cast<uint32_t>((i / depth) & 1);
+                    const long long start = clock64();
+                    while (!ptx::mbar_try_wait(bar, par)) {
+                        if (clock64() - start > p.timeout_cycles) {
+                            record_status(p.status, kStatusTimeout, kSiteTeardownLoads);
+                            break;
+                        }
                     }
                 }
-            }
+            };
+            drain(kStages, full_bar);
+            if constexpr (kSwap) drain(kSlots, sfull_bar);
         }
         __syncwarp();
     } else if (warp == 1) {
@@ -546,6 +575,35 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
         if constexpr (kPair) ptx::tmem_dealloc_pair(tmem_base, L::kTmemCols);
         else ptx::tmem_dealloc(tmem_base, L::kTmemCols);
     }
+    } else if (kSwap && warp == kPrepWarp) {
+    // ============================================================ scale preparation (swap mode)
+    // For each K-block, turn the slot's per-token scales sA[tok] into
+    // sA[tok] * sB, so the promotion does one FMA per element.
+    {
+        int sslot = 0;
+        uint32_t sphase = 0;
+        bool ok = true;
+        for (int t = t_first; ok && t < num_tiles; t += t_step) {
+            Tile tl;
+            if (!TM::decode(t, p, prefix, tl)) continue;
+            const int ncols = (tl.ntok + kTokBox - 1) / kTokBox * kTokBox;
+            for (int kb = kb_begin; kb < kb_end; ++kb) {
+                if (!wait(sfull_bar(sslot), sphase, kSitePromoFull)) { ok = false; break; }
+                float *sl = slots + sslot * L::kSlotFloats;
+                const float sb = sl[L::kScaleRows];
+                for (int j = lane; j < ncols; j += 32) sl[j] *= sb;
+                ptx::mbar_arrive(sready_bar(sslot));     // each lane: its own stores are released
+                if (++sslot == kSlots) { sslot = 0; sphase ^= 1u; }
+            }
+        }
+    }
+    if (clustered) {   // the promotion warps' two split-K cluster barriers
+        __syncwarp();
+        ptx::cluster_sync_all();
+        ptx::cluster_sync_all();
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
     } else {
     if constexpr (!kSwap) ptx::regs_inc<kRegsPromo>();
     // ============================================================ promotion
@@ -580,8 +638,8 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
     bool have_tile = false;
     int last_nvalid = 0;
     if (promo) {
-        int stage = 0, buf = 0;
-        uint32_t phase = 0, tphase = 0;
+        int stage = 0, buf = 0, sslot = 0;
+        uint32_t phase = 0, tphase = 0, sphase = 0;
         bool ok = true;
         for (int t = t_first; ok && t < num_tiles; t += t_step) {
             Tile tl;
@@ -595,10 +653,12 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
             const int nvalid = kSwap ? (ncols / kChunk - half + 1) / 2 : kChunks;
             const int wblk0 = tl.n0 / 128;
             for (int kb = kb_begin; kb < kb_end; ++kb) {
-                // the stage's scales: visible once its full barrier completed
-                if (!wait(full_bar(stage), phase, kSitePromoFull)) { ok = false; break; }
-                const float *slot = slots + stage * L::kSlotFloats;
-                float sa_row = 0.f, sb = 0.f;
+                // the K-block's scales: normal mode, visible once the stage's full
+                // barrier completed; swap mode, once the scale-prep warp is done
+                if (!wait(kSwap ? sready_bar(sslot) : full_bar(stage), kSwap ? sphase : phase,
+                          kSitePromoFull)) { ok = false; break; }
+                const float *slot = slots + (kSwap ? sslot : stage) * L::kSlotFloats;
+                float sa_row = 0.f;
                 float sbv[kNumSB];
                 if (!kSwap) {
                     sa_row = slot[lrow];
@@ -606,8 +666,6 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
                     for (int i = 0; i < kNumSB; ++i) sbv[i] = slot[L::kScaleRows + i];
                     __syncwarp();
                     if (lane == 0) ptx::mbar_arrive(empty_bar(stage));
-                } else {
-                    sb = slot[L::kScaleRows];
                 }
                 if (!wait(tfull_bar(buf), tphase, kSitePromoFull)) { ok = false; break; }
                 ptx::tc_fence_after();
@@ -705,19 +763,22 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
                             if (c == nvalid - 1) release_tmem(tempty_target);
                         }
                         float *a = acc + c * kChunk;
-                        // column (token) scales, broadcast from the slot
+                        // column (token) scales sA * sB, broadcast from the slot
                         const float4 *sc = reinterpret_cast<const float4 *>(slot + col_of(c));
 #pragma unroll
                         for (int i = 0; i < kChunk / 4; ++i) {
                             const float4 q4 = sc[i];
-                            ptx::ffma2s(a[4 * i + 0], a[4 * i + 1], q4.x * sb, q4.y * sb, v[4 * i + 0], v[4 * i + 1]);
-                            ptx::ffma2s(a[4 * i + 2], a[4 * i + 3], q4.z * sb, q4.w * sb, v[4 * i + 2], v[4 * i + 3]);
+                            a[4 * i + 0] = fmaf(q4.x, v[4 * i + 0], a[4 * i + 0]);
+                            a[4 * i + 1] = fmaf(q4.y, v[4 * i + 1], a[4 * i + 1]);
+                            a[4 * i + 2] = fmaf(q4.z, v[4 * i + 2], a[4 * i + 2]);
+                            a[4 * i + 3] = fmaf(q4.w, v[4 * i + 3], a[4 * i + 3]);
                         }
                     }
                 }
                 if (kSwap) {
                     __syncwarp();
-                    if (lane == 0) ptx::mbar_arrive(empty_bar(stage));
+                    if (lane == 0) ptx::mbar_arrive(sempty_bar(sslot));
+                    if (++sslot == kSlots) { sslot = 0; sphase ^= 1u; }
                 }
                 if (++stage == kStages) { stage = 0; phase ^= 1u; }
                 if (++buf == kAccBufs) { buf = 0; tphase ^= 1u; }
