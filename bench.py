@@ -132,6 +132,36 @@ class ClockSampler:
                 "sm_max_mhz": self.max_mhz, "reasons": reasons, "samples": len(self.samples)}
 
 
+# ----------------------------------------------------------------------------- multi-rank plumbing
+def rank_problem(workload: str, rank: int):
+    """The problem rank `rank` times: the named workload for rank 0, and for
+    other ranks the same shapes drawn from another seed (independent
+    problems, weak scaling; no data moves between ranks)."""
+    import workloads as W
+    if rank == 0:
+        return W.make_workload(workload)
+    spec = dict(W.WORKLOADS[workload])
+    spec["seed"] = spec["seed"] + 7919 * rank
+    kind = spec.pop("kind")
+    if kind == "dense":
+        return W.make_dense(**spec)
+    if kind == "contiguous":
+        return W.make_contiguous_multinomial(spec["G"], spec["tokens"], spec["N"], spec["K"], spec["seed"])
+    return W.make_masked_uniform(spec["G"], spec["Mmax"], spec["N"], spec["K"], spec["seed"])
+
+
+def max_over_ranks(values, device, world: int):
+    """Element-wise maximum of per-rank timings over all ranks (one small
+    all-reduce on the control path; nothing else crosses ranks)."""
+    if world <= 1:
+        return list(values)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor(list(values), device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
 # ----------------------------------------------------------------------------- our arm
 def run_ours(args, rank, world, local_rank):
     import numpy as np
@@ -144,18 +174,7 @@ def run_ours(args, rank, world, local_rank):
     dg_build.build()
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    prob = W.make_workload(args.workload)
-    if rank:
-        # independent problem per rank (same shapes, different values)
-        spec = dict(W.WORKLOADS[args.workload])
-        spec["seed"] = spec["seed"] + 7919 * rank
-        kind = spec.pop("kind")
-        if kind == "dense":
-            prob = W.make_dense(**spec)
-        elif kind == "contiguous":
-            prob = W.make_contiguous_multinomial(spec["G"], spec["tokens"], spec["N"], spec["K"], spec["seed"])
-        else:
-            prob = W.make_masked_uniform(spec["G"], spec["Mmax"], spec["N"], spec["K"], spec["seed"])
+    prob = rank_problem(args.workload, rank)
 
     host = {k: torch.from_numpy(np.ascontiguousarray(v)).pin_memory()
             for k, v in (("a", prob.a), ("sfa", prob.sfa), ("b", prob.b), ("sfb", prob.sfb))}
@@ -235,11 +254,7 @@ def run_ours(args, rank, world, local_rank):
     h2d = sum(v.numel() * v.element_size() for v in host.values())
     d2h = d.numel() * d.element_size()
 
-    # ---- max over ranks
-    if world > 1:
-        t = torch.tensor([ms, e2e_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms, e2e_ms = t.tolist()
+    ms, e2e_ms = max_over_ranks([ms, e2e_ms], dev, world)
     return prob, ms, e2e_ms, h2d, d2h, clocks
 
 
@@ -308,13 +323,12 @@ def cpu_baseline(prob, unit, budget_s=10.0):
 
 
 def run_reference(args, rank, world):
-    import workloads as W
     if rank != 0:
         return 0
-    prob = W.make_workload(args.workload)
+    prob = rank_problem(args.workload, 0)
     unit = UNIT[args.workload]
     # per-step CPU budget: the whole --steps/--warmup run stays within a few minutes
-    budget = max(0.2, min(6.0, 150.0 / max(1, args.steps + args.warmup)))
+    budget = max(0.2, min(2.0, 120.0 / max(1, args.steps + args.warmup)))
     for _ in range(args.warmup):
         cpu_baseline(prob, unit, budget_s=budget)
     vals = [cpu_baseline(prob, unit, budget_s=budget) for _ in range(args.steps)]

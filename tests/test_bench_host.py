@@ -1,0 +1,85 @@
+"""Host-side checks of bench.py: metric accounting, the reference (CPU
+oracle) arm, and the multi-rank plumbing on world_size-2 gloo process groups
+(no GPU needed)."""
+import json
+import os
+import socket
+import subprocess
+import sys
+
+import numpy as np
+import pytest
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+import bench  # noqa: E402
+import workloads as W  # noqa: E402
+
+
+def test_metric_value_units_and_world_scaling():
+    prob = W.Problem("dense", 64, 2112, 7168, 1, None, None, 0, None, None)
+    gbps = bench.metric_value(prob, "GB/s", 0.01, 1)
+    assert abs(gbps - prob.bytes() / 1e-5 / 1e9) < 1e-6
+    assert abs(bench.metric_value(prob, "GB/s", 0.01, 4) - 4 * gbps) < 1e-6
+    tf = bench.metric_value(prob, "TFLOP/s", 0.01, 2)
+    assert abs(tf - 2 * prob.flops() / 1e-5 / 1e12) < 1e-6
+
+
+def test_rank_problems_share_shapes_not_values():
+    p0, p1 = bench.rank_problem("dense_tiny", 0), bench.rank_problem("dense_tiny", 1)
+    assert p0.a.shape == p1.a.shape and p0.b.shape == p1.b.shape
+    assert not np.array_equal(p0.a, p1.a)
+
+
+def test_reference_arm_prints_one_json_line():
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--workload", "dense_tiny", "--steps", "1", "--warmup", "3"],
+                       cwd=ROOT, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr
+    lines = [l for l in r.stdout.splitlines() if l.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["cpu_baseline"]["kind"] == "oracle"
+    assert d["cpu_baseline"]["cores"] >= 1 and d["value"] > 0
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["unit"] == d["unit"]
+    assert d["config"]["workload"] == "dense_tiny"
+
+
+def test_reference_arm_other_ranks_exit_quietly():
+    env = dict(os.environ, RANK="1", WORLD_SIZE="2", LOCAL_RANK="1")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--workload", "dense_tiny", "--steps", "1", "--warmup", "3"],
+                       cwd=ROOT, env=env, capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0 and r.stdout.strip() == ""
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, q):
+    import torch.distributed as dist
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        got = bench.max_over_ranks([1.0 + rank, 5.0 - rank], "cpu", world)
+        q.put((rank, got))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_max_over_ranks_gloo_world_2():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(120)
+        assert p.exitcode == 0
+    res = dict(q.get(timeout=10) for _ in range(2))
+    assert res[0] == res[1] == [2.0, 5.0]
