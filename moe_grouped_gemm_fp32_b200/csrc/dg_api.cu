@@ -158,7 +158,7 @@ bool verbose() {
 template <int kBN, bool kSwap, int kStages, int kLayout, int kCtaGroup = 1>
 dg_status_t launch(const CUtensorMap &ma, const CUtensorMap &mb, const dg::Params &p, int grid_x,
                    int grid_y, int cluster_x, cudaStream_t stream) {
-    using L = dg::SmemLayout<kBN, kSwap, kStages, kCtaGroup>;
+    using L = dg::SmemLayout<kBN, kSwap, kStages, kCtaGroup, kSwap && kLayout == dg::kDense && kBN <= 128>;
     auto kernel = dg::fp8_gemm_kernel<kBN, kSwap, kStages, kLayout, kCtaGroup>;
     static bool attr_done[kMaxDevices] = {};
     int dev = 0;
@@ -213,7 +213,7 @@ dg_status_t launch(const CUtensorMap &ma, const CUtensorMap &mb, const dg::Param
 // (cached per device and cluster size).  0 if the query fails.
 template <int kBN, bool kSwap, int kStages, int kLayout, int kCtaGroup = 1>
 int max_active_clusters(int cluster_x) {
-    using L = dg::SmemLayout<kBN, kSwap, kStages, kCtaGroup>;
+    using L = dg::SmemLayout<kBN, kSwap, kStages, kCtaGroup, kSwap && kLayout == dg::kDense && kBN <= 128>;
     auto kernel = dg::fp8_gemm_kernel<kBN, kSwap, kStages, kLayout, kCtaGroup>;
     static int cache[kMaxDevices][9] = {};
     int dev = 0;
@@ -245,21 +245,18 @@ int max_active_clusters(int cluster_x) {
     return n;
 }
 
-// Split-K factor for swap-mode tiles: the largest power of two <= 8 such that
-// every cluster of the grid is resident at once (one wave), each CTA keeps at
-// least two K-blocks, and the CTAs fit on the SMs.  DG_SPLIT_K overrides it
-// (tuning sweeps).
-template <int kBN, int kLayout>
+// Split-K factor for swap-mode tiles: the largest split <= 8 such that every
+// cluster of the grid is resident at once (one wave), each CTA keeps at least
+// two K-blocks, and the CTAs fit on the SMs.  DG_SPLIT_K overrides it (tuning).
+template <int kBN, int kStages, int kLayout>
 int choose_split(int tiles, int num_kb, int num_sms) {
     static int forced = [] {
         const char *s = std::getenv("DG_SPLIT_K");
         return s ? std::atoi(s) : 0;
     }();
-    if (forced == 1 || forced == 2 || forced == 4 || forced == 8)
-        return num_kb >= forced ? forced : 1;
-    for (int split = 8; split >= 2; split /= 2) {
+    if (forced >= 1 && forced <= 8) return num_kb >= 2 * forced ? forced : 1;
+    for (int split = 8; split >= 2; --split) {
         if (tiles * split > num_sms || num_kb < 2 * split) continue;
-        constexpr int kStages = kBN == 64 ? 8 : (kBN == 128 ? 6 : 4);
         if (max_active_clusters<kBN, true, kStages, kLayout>(split) >= tiles) return split;
     }
     return 1;
@@ -305,15 +302,15 @@ dg_status_t dg_fp8_gemm_nt(const uint8_t *a, const float *sfa, int ld_sfa, const
         // swap-AB: weights on the 128 TMEM lanes, the few tokens on the MMA's N side
         const int bn = M <= 64 ? 64 : (M <= 128 ? 128 : 256);
         const int tiles = ((N + 127) / 128) * ((M + bn - 1) / bn);
-        p.split = bn == 64    ? choose_split<64, dg::kDense>(tiles, p.num_kb, info->num_sms)
-                  : bn == 128 ? choose_split<128, dg::kDense>(tiles, p.num_kb, info->num_sms)
-                              : choose_split<256, dg::kDense>(tiles, p.num_kb, info->num_sms);
+        p.split = bn == 64    ? choose_split<64, 7, dg::kDense>(tiles, p.num_kb, info->num_sms)
+                  : bn == 128 ? choose_split<128, 4, dg::kDense>(tiles, p.num_kb, info->num_sms)
+                              : 1;   // 256-token tiles run persistent (no split-K buffer)
         if ((st = make_map(&mb, b, K, N, 1, 128)) != DG_SUCCESS) return st;
         if ((st = make_map(&ma, a, K, M, 1, 32)) != DG_SUCCESS) return st;   // 32-token boxes
         const int gx = p.split > 1 ? p.split : (tiles < info->num_sms ? tiles : info->num_sms);
         const int gy = p.split > 1 ? tiles : 1;
-        if (bn == 64) return launch<64, true, 8, dg::kDense>(ma, mb, p, gx, gy, p.split, s);
-        if (bn == 128) return launch<128, true, 6, dg::kDense>(ma, mb, p, gx, gy, p.split, s);
+        if (bn == 64) return launch<64, true, 7, dg::kDense>(ma, mb, p, gx, gy, p.split, s);
+        if (bn == 128) return launch<128, true, 4, dg::kDense>(ma, mb, p, gx, gy, p.split, s);
         return launch<256, true, 4, dg::kDense>(ma, mb, p, gx, gy, p.split, s);
     }
     if (N <= 128) {

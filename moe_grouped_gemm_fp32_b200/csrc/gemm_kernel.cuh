@@ -231,7 +231,7 @@ struct TileMap {
     }
 };
 
-template <int kBN, bool kSwap, int kStages, int kCtaGroup>
+template <int kBN, bool kSwap, int kStages, int kCtaGroup, bool kSplitK = false>
 struct SmemLayout {
     static constexpr int kYRows = kSwap ? kBN : kBN / kCtaGroup;   // rows of the Y operand per CTA
     static constexpr int kXBytes = kTileX * kBlockK;               // 16 KB
@@ -257,18 +257,24 @@ struct SmemLayout {
     static constexpr int kMiscOffset = kBarOffset + kNumBars * 8;     // tmem addr, abort flag
     static constexpr int kPrefixOffset = (kMiscOffset + 16 + 15) / 16 * 16;
     static constexpr int kPrefixBytes = (kMaxGroups + 1) * 4;
-    static constexpr int kUsed = kPrefixOffset + kPrefixBytes;
+    // split-K receive buffer: [source rank][owned row][column], rows padded by
+    // 4 floats (bank spread); 136 rows cover any split of 128 rows into <= 8 owners
+    static constexpr int kRecvStride = kBN + 4;
+    static constexpr int kRecvRows = 136;
+    static constexpr int kRecvOffset = (kPrefixOffset + kPrefixBytes + 127) / 128 * 128;
+    static constexpr int kRecvBytes = kSplitK ? kRecvRows * kRecvStride * 4 : 0;
+    static constexpr int kUsed = kRecvOffset + kRecvBytes;
     static constexpr int kAlloc = (kUsed + 1024 > kMinSmem) ? kUsed + 1024 : kMinSmem;
     static constexpr int kTmemCols = kAccBufs * kBN <= 32    ? 32
                                      : kAccBufs * kBN <= 64  ? 64
                                      : kAccBufs * kBN <= 128 ? 128
                                      : kAccBufs * kBN <= 256 ? 256 : 512;
     static_assert(kAccBufs * kBN <= 512, "TMEM holds 512 columns");
-    static constexpr int kRecvStride = kBN + 4;   // split-K receive rows, padded (bank spread)
     static_assert(kStageBytes % 1024 == 0, "stage must keep 1024-byte alignment");
-    static_assert(kSlotBytes % 16 == 0, "bulk copies need 16-byte aligned slots");
-    static_assert(!kSwap || kStagesBytes >= kTileX * kRecvStride * 4,
-                  "split-K receive buffer reuses the stages");
+    static_assert(kSlotBytes % 16 == 0 && kSlotOffset % 16 == 0, "bulk copies need 16-byte aligned slots");
+    static_assert(kBarOffset % 8 == 0, "mbarriers are 8-byte objects");
+    static_assert(kPrefixOffset % 16 == 0, "prefix table alignment");
+    static_assert(kRecvOffset % 16 == 0, "split-K pushes and reads are 16-byte vectors");
     static_assert(kAlloc <= 227 * 1024, "shared memory budget");
 };
 
@@ -276,7 +282,12 @@ template <int kBN, bool kSwap, int kStages, int kLayout, int kCtaGroup>
 __global__ void __launch_bounds__(num_threads(kSwap), 1)
 fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                 const Params p) {
-    using L = SmemLayout<kBN, kSwap, kStages, kCtaGroup>;
+    // dense swap-mode kernels may run split-K (one tile per cluster)
+    constexpr bool kSplitK = kSwap && kLayout == kDense && kBN <= 128;
+    // the producer starts loading before the set-up barrier when nothing it
+    // needs comes from other warps (not for CTA pairs or the masked layout)
+    constexpr bool kEarly = kCtaGroup == 1 && kLayout != kMasked;
+    using L = SmemLayout<kBN, kSwap, kStages, kCtaGroup, kSplitK>;
     using TM = TileMap<kBN, kSwap, kLayout, kCtaGroup>;
     static_assert(kBN == 64 || kBN == 128 || kBN == 160 || kBN == 224 || kBN == 256, "tile N");
     static_assert(kCtaGroup == 1 || (kCtaGroup == 2 && !kSwap && kLayout == kDense),
@@ -380,13 +391,20 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
         }
     }
     ptx::tc_fence_before();
-    __syncthreads();
+    if constexpr (kEarly) {
+        // warp 0 (the producer; thread 0 initialised the barriers) arrives and
+        // goes on; the other warps wait until the barriers and TMEM are ready
+        if (warp == 0) ptx::named_bar_arrive(1, num_threads(kSwap));
+        else ptx::named_bar_sync(1, num_threads(kSwap));
+    } else {
+        __syncthreads();
+    }
     if constexpr (kPair) ptx::cluster_sync_all();   // the peer's barriers exist before any remote use
     ptx::tc_fence_after();
-    const uint32_t tmem_base = *tmem_slot;
+    const uint32_t tmem_base = warp == 0 && kEarly ? 0u : *tmem_slot;
 
     // tile iteration: persistent (split == 1) or one tile per cluster (split > 1)
-    const bool clustered = kSwap && kLayout == kDense && p.split > 1;   // split-K is a dense swap-mode path
+    const bool clustered = kSplitK && p.split > 1;   // split-K: dense swap-mode path
     const int num_tiles = clustered ? static_cast<int>(gridDim.y) : TM::count(p, prefix);
     const int t_first = clustered ? static_cast<int>(blockIdx.y) : static_cast<int>(blockIdx.x) / kCtaGroup;
     const int t_step = clustered ? num_tiles : static_cast<int>(gridDim.x) / kCtaGroup;
@@ -407,6 +425,9 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
     if constexpr (!kSwap) ptx::regs_dec<kRegsIssue>();
     if (warp == 0) {
         // ======================================================== producer
+        // (one elected thread; the warp-wide sync orders it after thread 0's
+        // barrier initialisation when the producer starts before the set-up barrier)
+        __syncwarp();
         if (ptx::elect_one()) {
             int stage = 0, sslot = 0;
             uint32_t phase = 0, sphase = 0;
@@ -548,9 +569,8 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
         __syncwarp();
     }
 
-    if (clustered) {   // the promotion warps' two split-K cluster barriers
+    if (clustered) {   // the split-K exchange barrier of the promotion warps
         __syncwarp();
-        ptx::cluster_sync_all();
         ptx::cluster_sync_all();
     }
     // ------------------------------------------------------------ teardown (issue warps)
@@ -597,9 +617,8 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
             }
         }
     }
-    if (clustered) {   // the promotion warps' two split-K cluster barriers
+    if (clustered) {   // the split-K exchange barrier of the promotion warps
         __syncwarp();
-        ptx::cluster_sync_all();
         ptx::cluster_sync_all();
     }
     ptx::tc_fence_before();
@@ -832,17 +851,17 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
 
     // ============================================================ split-K reduction
     if (clustered) {
-        // (1) every CTA of the cluster is done with its main loop: stage memory is idle
-        __syncwarp();
-        ptx::cluster_sync_all();
+        // (1) push this thread's row to its owner's receive buffer, slot
+        // [source rank][owned row][column].  The buffer is private to the split-K
+        // exchange, so no CTA waits for the others before writing.
         const int split = p.split;
-        const int rows_per = kTileX / split;             // split divides 128 (1,2,4,8)
+        const int rows_per = (kTileX + split - 1) / split;     // the last owner may get fewer
         const uint32_t my_rank = ptx::cluster_rank();
-        if (promo && have_tile && !*abort_flag) {
-            // (2) send this thread's row to its owner: slot [src rank][row % rows_per][column]
+        const uint32_t recv_base = s_base + L::kRecvOffset;
+        if (have_tile && !*abort_flag) {
             const int owner = lrow / rows_per;
-            const uint32_t local = s_base + static_cast<uint32_t>(
-                ((my_rank * rows_per + (lrow % rows_per)) * L::kRecvStride) * 4);
+            const uint32_t local = recv_base + static_cast<uint32_t>(
+                ((my_rank * rows_per + (lrow - owner * rows_per)) * L::kRecvStride) * 4);
             const uint32_t remote = ptx::map_cluster(local, static_cast<uint32_t>(owner));
 #pragma unroll
             for (int c = 0; c < kChunks; ++c) {
@@ -855,22 +874,25 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
                 }
             }
         }
+        // (2) every push of the cluster has landed
+        __syncwarp();
         ptx::cluster_sync_all();
         // (3) each CTA sums its rows over the source ranks in rank order and stores.
         // Thread -> (row rr, 4 columns j4): consecutive threads take consecutive rows,
         // so a quarter-warp's 16-byte reads hit distinct banks (padded row stride)
         // and a warp's BF16 stores of one column are contiguous in D.
-        if (promo && have_tile) {
-            const float4 *recv = reinterpret_cast<const float4 *>(smem);
+        if (have_tile) {
+            const float4 *recv = reinterpret_cast<const float4 *>(smem + L::kRecvOffset);
             const Tile &tl = last_tile;
             const size_t row_base = kLayout == kMasked ? static_cast<size_t>(tl.g) * p.M : 0;
             const int tid = (warp - kPromoWarp0) * 32 + lane;        // 0..255
+            const int my_rows = min(rows_per, kTileX - static_cast<int>(my_rank) * rows_per);
             const int groups = (tl.ntok + 3) / 4;
-            const int elems = rows_per * groups;
+            const int elems = my_rows > 0 ? my_rows * groups : 0;
             const int n = tl.n0 + static_cast<int>(my_rank) * rows_per;
             for (int e = tid; e < elems; e += 256) {
-                const int rr = e % rows_per;
-                const int j4 = e / rows_per;
+                const int rr = e % my_rows;
+                const int j4 = e / my_rows;
                 float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
                 for (int src = 0; src < split; ++src) {
                     const float4 v = recv[((src * rows_per + rr) * L::kRecvStride) / 4 + j4];
