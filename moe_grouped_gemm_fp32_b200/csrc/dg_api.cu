@@ -262,6 +262,16 @@ int choose_split(int tiles, int num_kb, int num_sms) {
     return 1;
 }
 
+// Efficiency of a pair-tile width: the share of the tiles' columns that are
+// real (N tail) times how full the waves of resident pairs are.
+double pair_efficiency(long long rows_pairs, int N, int bn, int pairs_max) {
+    if (pairs_max <= 0) return 0.0;
+    const long long nt = (N + bn - 1) / bn;
+    const long long tiles = rows_pairs * nt;
+    const long long waves = (tiles + pairs_max - 1) / pairs_max;
+    return (static_cast<double>(N) / (nt * bn)) * (static_cast<double>(tiles) / (waves * pairs_max));
+}
+
 dg::Params base_params(const float *sfa, int ld_sfa, const float *sfb, void *d, int rows, int N,
                        int K, int G, const DeviceInfo *info) {
     dg::Params p = {};
@@ -326,10 +336,14 @@ dg_status_t dg_fp8_gemm_nt(const uint8_t *a, const float *sfa, int ld_sfa, const
         const char *e = std::getenv("DG_PAIR_N");
         return e ? std::atoi(e) : 0;
     }();
-    const int bn = (forced_bn == 160 || forced_bn == 224 || forced_bn == 256) ? forced_bn : 224;
+    const long long row_pairs = (M + 255) / 256;
+    const int pm224 = max_active_clusters<224, false, 6, dg::kDense, 2>(2);
+    const int pm256 = max_active_clusters<256, false, 6, dg::kDense, 2>(2);
+    int bn = pair_efficiency(row_pairs, N, 224, pm224) > pair_efficiency(row_pairs, N, 256, pm256) + 1e-9
+                 ? 224 : 256;
+    if (forced_bn == 160 || forced_bn == 224 || forced_bn == 256) bn = forced_bn;
     const int pairs_max = bn == 160   ? max_active_clusters<160, false, 7, dg::kDense, 2>(2)
-                          : bn == 224 ? max_active_clusters<224, false, 6, dg::kDense, 2>(2)
-                                      : max_active_clusters<256, false, 6, dg::kDense, 2>(2);
+                          : bn == 224 ? pm224 : pm256;
     if (pairs_max <= 0) return cuda_fail(cudaErrorInvalidConfiguration, "no resident CTA pair");
     const int tiles = ((M + 255) / 256) * ((N + bn - 1) / bn);
     const int pairs = tiles < pairs_max ? tiles : pairs_max;
@@ -354,10 +368,35 @@ dg_status_t dg_m_grouped_fp8_gemm_nt_contiguous(const uint8_t *a, const float *s
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     dg::Params p = base_params(sfa, ld_sfa, sfb, d, M_total, N, K, G, info);
     p.m_indices = m_indices;
+    CUtensorMap ma, mb;
+    // CTA pairs for the contiguous layout measured no faster than 128 x 256
+    // single-CTA tiles on the 4-group workload (both are bound by the MMA /
+    // promotion hand-off, not by operand traffic); DG_CONTIG_PAIRS=1 selects them.
+    static const bool contig_pairs = [] {
+        const char *e = std::getenv("DG_CONTIG_PAIRS");
+        return e && e[0] == '1';
+    }();
+    if (contig_pairs && N > 128 && G < dg::kMaxGroups) {
+        // CTA pairs with 256-row tiles; pairs straddling a group boundary run
+        // a second pass (the tile count grows by at most (G-1) x N-tiles)
+        const long long row_pairs = (M_total / 128 + 1) / 2;
+        const int pm224 = max_active_clusters<224, false, 6, dg::kContiguous, 2>(2);
+        const int pm256 = max_active_clusters<256, false, 6, dg::kContiguous, 2>(2);
+        const int bn = pair_efficiency(row_pairs, N, 224, pm224) > pair_efficiency(row_pairs, N, 256, pm256) + 1e-9
+                           ? 224 : 256;
+        const int pairs_max = bn == 224 ? pm224 : pm256;
+        if (pairs_max > 0) {
+            const long long tiles = row_pairs * ((N + bn - 1) / bn);
+            const int pairs = tiles < pairs_max ? static_cast<int>(tiles) : pairs_max;
+            if ((st = make_map(&ma, a, K, M_total, 1, 128)) != DG_SUCCESS) return st;
+            if ((st = make_map(&mb, b, K, N, G, bn / 2)) != DG_SUCCESS) return st;
+            if (bn == 224) return launch<224, false, 6, dg::kContiguous, 2>(ma, mb, p, 2 * pairs, 1, 2, s);
+            return launch<256, false, 6, dg::kContiguous, 2>(ma, mb, p, 2 * pairs, 1, 2, s);
+        }
+    }
     const int bn = N <= 128 ? 128 : 256;
     const int tiles = (M_total / 128) * ((N + bn - 1) / bn);
     const int grid = tiles < info->num_sms ? tiles : info->num_sms;
-    CUtensorMap ma, mb;
     if ((st = make_map(&ma, a, K, M_total, 1, 128)) != DG_SUCCESS) return st;
     if ((st = make_map(&mb, b, K, N, G, bn)) != DG_SUCCESS) return st;
     if (bn == 128) return launch<128, false, 6, dg::kContiguous>(ma, mb, p, grid, 1, 1, s);

@@ -158,6 +158,7 @@ struct Tile {
     int tok_end; // exclusive bound of valid token rows
     int n0;      // first weight row
     int ntok;    // token rows of this tile that exist: min(rows per tile, tok_end - tok0)
+    int store;   // CTA-pair tiles: bit r set = CTA r of the pair stores its rows
 };
 
 template <int kBN, bool kSwap, int kLayout, int kCtaGroup>
@@ -166,10 +167,27 @@ struct TileMap {
     static constexpr int kWRows = kSwap ? kTileX : kBN;                // weight rows per tile
     static constexpr int kRasterM = 16 / kCtaGroup;                    // L2 raster band (token blocks)
 
+    // Contiguous layout in CTA pairs: a pair tile covers two 128-row blocks.
+    // When the two blocks belong to different groups, the tile runs twice: the
+    // first pass (group of block 0) stores block 0's rows, a second pass (group
+    // of block 1), listed after all first passes, stores block 1's rows.  The
+    // pairs that need a second pass are listed in prefix[0..Q), Q in
+    // prefix[kMaxGroups] (built at kernel set-up).
+    static constexpr bool kPairedGroups = kLayout == kContiguous && kCtaGroup == 2;
+    __device__ static int block_group(const Params &p, int blk) {
+        if (blk >= p.M / kTileX) return -1;
+        const int g = __ldg(p.m_indices + static_cast<size_t>(blk) * kTileX);
+        return g < p.G ? g : -1;
+    }
+
     // Number of tiles (masked: from the smem prefix table).
     __device__ static int count(const Params &p, const int *prefix) {
         const int nw = (p.N + kWRows - 1) / kWRows;
         if (kLayout == kMasked) return prefix[p.G];
+        if (kPairedGroups) {
+            const int npairs = (p.M / kTileX + 1) / 2;
+            return (npairs + prefix[kMaxGroups]) * nw;
+        }
         const int nt = (p.M + kTokRows - 1) / kTokRows;
         return nt * nw;
     }
@@ -199,6 +217,40 @@ struct TileMap {
             tl.tok_end = mm;
             tl.n0 = wb * kWRows;
             tl.ntok = min(kTokRows, mm - tl.tok0);
+            tl.store = 3;
+            return true;
+        }
+        if (kPairedGroups) {
+            const int npairs = (p.M / kTileX + 1) / 2;
+            const int first = npairs * nw;
+            int pair, g, store;
+            if (t < first) {
+                const int per_band = kRasterM * nw;
+                const int band = t / per_band;
+                const int b0 = band * kRasterM;
+                const int width = min(kRasterM, npairs - b0);
+                const int local = t - band * per_band;
+                pair = b0 + local % width;
+                wb = local / width;
+                const int g0 = block_group(p, 2 * pair), g1 = block_group(p, 2 * pair + 1);
+                g = g0 >= 0 ? g0 : g1;
+                if (g < 0) return false;
+                store = (g0 == g ? 1 : 0) | (g1 == g ? 2 : 0);
+            } else {
+                const int q = (t - first) / nw;
+                wb = t - first - q * nw;
+                pair = prefix[q];
+                g = block_group(p, 2 * pair + 1);
+                store = 2;
+            }
+            tl.g = g;
+            tl.tok0 = pair * kTokRows;
+            tl.a_row = tl.tok0;
+            tl.a_grp = 0;
+            tl.tok_end = p.M;
+            tl.n0 = wb * kWRows;
+            tl.ntok = min(kTokRows, p.M - tl.tok0);
+            tl.store = store;
             return true;
         }
         const int nt = (p.M + kTokRows - 1) / kTokRows;
@@ -221,6 +273,7 @@ struct TileMap {
         tl.n0 = wb * kWRows;
         tl.ntok = min(kTokRows, p.M - tl.tok0);
         tl.g = 0;
+        tl.store = 3;
         if (kLayout == kContiguous) {
             const int g = __ldg(p.m_indices + tl.tok0);
             if (g < 0) return false;
@@ -290,8 +343,8 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
     using L = SmemLayout<kBN, kSwap, kStages, kCtaGroup, kSplitK>;
     using TM = TileMap<kBN, kSwap, kLayout, kCtaGroup>;
     static_assert(kBN == 64 || kBN == 128 || kBN == 160 || kBN == 224 || kBN == 256, "tile N");
-    static_assert(kCtaGroup == 1 || (kCtaGroup == 2 && !kSwap && kLayout == kDense),
-                  "CTA pairs: dense normal mode");
+    static_assert(kCtaGroup == 1 || (kCtaGroup == 2 && !kSwap && kLayout != kMasked),
+                  "CTA pairs: dense or contiguous, normal mode");
     constexpr bool kPair = kCtaGroup == 2;
     constexpr int kHalf = kBN / 2;               // columns per promotion warpgroup
     constexpr int kChunk = kHalf > 64 ? 16 : 32; // TMEM columns per load (register budget)
@@ -380,6 +433,31 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
             carry += __shfl_sync(0xffffffffu, incl, 31);
         }
         if (lane == 0) prefix[p.G] = carry;
+    }
+    if (TM::kPairedGroups && warp == kPromoWarp0) {
+        // pairs of 128-row blocks whose groups differ: they get a second pass
+        const int nblk = p.M / kTileX, npairs = (nblk + 1) / 2;
+        int count = 0;
+        for (int base = 0; base < npairs; base += 32) {
+            const int pr = base + lane;
+            bool second = false;
+            if (pr < npairs) {
+                for (int b = 2 * pr; b <= 2 * pr + 1 && b < nblk; ++b)
+                    if (__ldg(p.m_indices + static_cast<size_t>(b) * kTileX) >= p.G)
+                        record_status(p.status, kStatusInvalid, kSiteBadGroup);
+                const int g0 = TM::block_group(p, 2 * pr), g1 = TM::block_group(p, 2 * pr + 1);
+                second = g0 >= 0 && g1 >= 0 && g0 != g1;
+            }
+            const unsigned ballot = __ballot_sync(0xffffffffu, second);
+            const int slot = count + __popc(ballot & ((1u << lane) - 1u));
+            if (second && slot < kMaxGroups) prefix[slot] = pr;
+            count += __popc(ballot);
+        }
+        if (count > kMaxGroups) {
+            if (lane == 0) record_status(p.status, kStatusInvalid, kSiteBadGroup);
+            count = kMaxGroups;
+        }
+        if (lane == 0) prefix[kMaxGroups] = count;
     }
     if (warp == 1) {
         if constexpr (kPair) {
@@ -653,7 +731,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
             else ptx::mbar_arrive(target);
         }
     };
-    Tile last_tile{0, 0, 0, 0, 0, 0, 0};
+    Tile last_tile{0, 0, 0, 0, 0, 0, 0, 3};
     bool have_tile = false;
     int last_nvalid = 0;
     if (promo) {
@@ -666,7 +744,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
 #pragma unroll
             for (int i = 0; i < kHalf; ++i) acc[i] = 0.f;
             const int my_tok = tl.tok0 + my_row0 + lrow;   // normal mode: this thread's token row
-            const bool tok_ok = my_tok < tl.tok_end;
+            const bool tok_ok = my_tok < tl.tok_end && ((tl.store >> pair_rank) & 1);
             // chunks of this warpgroup that hold columns of the tile
             const int ncols = kSwap ? (tl.ntok + kTokBox - 1) / kTokBox * kTokBox : kBN;
             const int nvalid = kSwap ? (ncols / kChunk - half + 1) / 2 : kChunks;

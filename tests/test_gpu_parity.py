@@ -101,9 +101,31 @@ def test_dense_deterministic():
 # ------------------------------------------------------------------ contiguous
 @pytest.mark.parametrize("counts,N,K", [([130, 0, 700, 5], 384, 512),
                                         ([0, 0, 1, 0], 256, 256),
-                                        ([128, 256], 2112, 512)])
+                                        ([128, 256], 2112, 512),
+                                        # 128-row blocks 4|5 and 2|3 of different groups share a
+                                        # CTA pair tile (second pass), odd block count at the end
+                                        ([130, 200, 5, 300, 129], 448, 384),
+                                        ([1, 1, 1, 1, 1, 1, 1], 256, 256)])
 def test_contiguous(counts, N, K):
     _run_full(W.make_contiguous(counts, N, K, seed=sum(counts) + N))
+
+
+@pytest.mark.parametrize("counts,N,K", [([130, 200, 5, 300, 129], 448, 384), ([128, 256], 2112, 512)])
+def test_contiguous_cta_pairs(counts, N, K):
+    """The CTA-pair contiguous path (opt-in) in a child process: second passes
+    for pair tiles whose two 128-row blocks belong to different groups."""
+    import os, subprocess, sys
+    code = ("import sys; sys.path[:0] = [%r, %r]\n"
+            "import workloads as W, oracle\n"
+            "from gpu_util import DeviceProblem, compare, to_f64, valid_mask\n"
+            "p = W.make_contiguous(%r, %d, %d, seed=77)\n"
+            "dp = DeviceProblem(p); dp.fill_sentinel(); d = to_f64(dp.run())\n"
+            "compare(d, oracle.solve(p), valid_mask(p)); print('OK')\n"
+            % (os.path.dirname(os.path.dirname(__file__)), os.path.dirname(__file__), counts, N, K))
+    env = dict(os.environ, DG_CONTIG_PAIRS="1", DG_VERBOSE="1")
+    r = subprocess.run([sys.executable, "-c", code], env=env, capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0 and "OK" in r.stdout, r.stdout + r.stderr
+    assert "ctas/mma=2" in r.stderr
 
 
 def test_contiguous_multinomial_small():
