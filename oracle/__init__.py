@@ -55,6 +55,10 @@ def _load():
         for f in ("oracle_fp8_gemm_nt", "oracle_m_grouped_contiguous",
                   "oracle_m_grouped_masked", "oracle_points"):
             getattr(lib, f).restype = ctypes.c_int
+        lib.oracle_e4m3_encode.argtypes = [ctypes.c_float]
+        lib.oracle_e4m3_encode.restype = ctypes.c_uint8
+        lib.oracle_quantize_1x128.argtypes = [P, L, L, P, P, L]
+        lib.oracle_quantize_1x128.restype = ctypes.c_int
         _lib = lib
     return _lib
 
@@ -142,3 +146,24 @@ def solve(prob) -> np.ndarray:
                                prob.m_indices, prob.M, prob.N, prob.K, prob.G)
     return gemm_masked(prob.a, prob.sfa, prob.ld_sfa, prob.b, prob.sfb, prob.masked_m,
                        prob.G, prob.M, prob.N, prob.K)
+
+
+def e4m3_encode(values) -> np.ndarray:
+    """The oracle's E4M3 round-to-nearest-even encoder, element by element."""
+    lib = _load()
+    v = np.asarray(values, dtype=np.float32).ravel()
+    return np.array([lib.oracle_e4m3_encode(float(x)) for x in v], dtype=np.uint8)
+
+
+def quantize_1x128(x: np.ndarray, ld_sfa: Optional[int] = None):
+    """Per-token 1x128 quantisation of float32 x [M, K] (the exact BF16 inputs):
+    returns (q uint8 [M, K], sfa float32 [KB, ld_sfa])."""
+    x = _c(x, np.float32)
+    M, K = x.shape
+    ld = ld_sfa if ld_sfa is not None else (M + 3) // 4 * 4
+    q = np.empty((M, K), dtype=np.uint8)
+    sfa = np.zeros((K // 128, ld), dtype=np.float32)
+    rc = _load().oracle_quantize_1x128(_p(x), M, K, _p(q), _p(sfa), ld)
+    if rc:
+        raise ValueError(f"oracle_quantize_1x128 rejected the shape (rc={rc})")
+    return q, sfa

@@ -203,3 +203,78 @@ int oracle_points(int layout, const uint8_t *a, const float *sfa, long ld_sfa,
     }
     return 0;
 }
+
+/* ------------------------------------------------------------------------
+ * Per-token 1x128 activation quantiser (the step that produces A and sA;
+ * DeepGEMM page 2 "技术特性": fine-grained scaling, each small block with its
+ * own scale; page 3 "精细粒度缩放": block-wise instead of tensor-wise).
+ *
+ * For row m and K-block kb of x [M][K] (values given as FP32, the exact BF16
+ * inputs widened):
+ *   amax = max |x[m, kb*128 .. kb*128+127]|          (exact)
+ *   s    = fl32(amax / 448), or 1 when amax == 0     (one FP32 rounding)
+ *   q    = E4M3_RNE(clamp(fl32(x / s), -448, 448))   (FP32 division, then RNE)
+ * s is stored at sfa[kb * ld_sfa + m] (MN-major), q at q[m * K + k].
+ * ------------------------------------------------------------------------ */
+
+/* Round a finite float to the nearest E4M3 ("fn") value, ties to even; the
+ * input must already lie in [-448, 448].  From the bit-field definition: a
+ * value with exponent e >= -6 has 3 fraction bits (spacing 2^(e-3)); below
+ * 2^-6 the spacing is the subnormal step 2^-9. */
+uint8_t oracle_e4m3_encode(float x)
+{
+    uint8_t sign = (x < 0.0f || (x == 0.0f && signbit(x))) ? 0x80 : 0x00;
+    double a = fabs((double)x);
+    if (a == 0.0) return sign;
+    int e;
+    frexp(a, &e);                 /* a = f * 2^e, f in [0.5, 1) -> exponent e-1 */
+    int exp2 = e - 1;
+    if (exp2 < -6) exp2 = -6;     /* subnormal range: fixed spacing 2^-9 */
+    double spacing = ldexp(1.0, exp2 - 3);
+    double units = a / spacing;   /* exact: a power-of-two rescale */
+    double lo = floor(units);
+    double frac = units - lo;
+    double r = lo;
+    if (frac > 0.5 || (frac == 0.5 && fmod(lo, 2.0) != 0.0)) r = lo + 1.0;
+    if (r == 0.0) return sign;    /* rounds to a signed zero */
+    double v = r * spacing;       /* may carry into the next binade: still exact */
+    /* encode v (0 < v <= 448) */
+    int ve;
+    frexp(v, &ve);
+    int vexp = ve - 1;
+    uint8_t code;
+    if (vexp < -6) {
+        code = (uint8_t)(v / ldexp(1.0, -9));                 /* subnormal mantissa */
+    } else {
+        int mant = (int)((v / ldexp(1.0, vexp) - 1.0) * 8.0);
+        code = (uint8_t)(((vexp + 7) << 3) | mant);
+    }
+    return (uint8_t)(sign | code);
+}
+
+int oracle_quantize_1x128(const float *x, long M, long K, uint8_t *q, float *sfa, long ld_sfa)
+{
+    if (M < 0 || K <= 0 || K % ORC_BLOCK != 0 || ld_sfa < M) return 1;
+    long KB = K / ORC_BLOCK;
+    #pragma omp parallel for schedule(static)
+    for (long m = 0; m < M; ++m) {
+        for (long kb = 0; kb < KB; ++kb) {
+            const float *xb = x + m * K + kb * ORC_BLOCK;
+            float amax = 0.0f;
+            for (int i = 0; i < ORC_BLOCK; ++i) {
+                float v = fabsf(xb[i]);
+                if (v > amax) amax = v;
+            }
+            float s = amax / 448.0f;
+            if (amax == 0.0f) s = 1.0f;
+            sfa[kb * ld_sfa + m] = s;
+            for (int i = 0; i < ORC_BLOCK; ++i) {
+                float t = xb[i] / s;
+                if (t > 448.0f) t = 448.0f;
+                if (t < -448.0f) t = -448.0f;
+                q[m * K + kb * ORC_BLOCK + i] = oracle_e4m3_encode(t);
+            }
+        }
+    }
+    return 0;
+}
