@@ -4,7 +4,9 @@
 
 One step = one call of the hot path (scheduling, TMA loads, tcgen05 MMA,
 per-K-block promotion, epilogue; swap-AB and split-K for small M) on one
-batch of seeded synthetic inputs already resident in HBM.  L2 is flushed
+batch of seeded synthetic inputs already resident in HBM.  The ``quant_*``
+workloads time the per-token 1x128 activation quantiser that produces the
+GEMM's A operand instead (GB/s of BF16 in + E4M3 and scales out).  L2 is flushed
 before every timed step (a 512 MB write, then a 256 MB read so that no dirty
 line of the flush is left to write back during the step) and the step is
 timed alone with CUDA events on the launching stream.  Multi-GPU (torchrun): each rank runs its own
@@ -35,16 +37,30 @@ DEFAULT_WORKLOAD = "dense_decode_m64"
 # context only).  DeepGEMM page 2 "性能实测": M=64 N=2112 K=7168 -> 1688 GB/s.
 PAGES_NUMBER = {"dense_decode_m64": (1688.0, "GB/s")}
 UNIT = {"dense_tiny": "TFLOP/s", "dense_decode_m64": "GB/s", "dense_decode_m128": "GB/s",
-        "dense_large": "TFLOP/s", "contiguous_g4": "TFLOP/s", "masked_g16": "GB/s"}
-KERNEL_SOURCES = ["moe_grouped_gemm_fp32_b200/csrc/gemm_kernel.cuh",
-                  "moe_grouped_gemm_fp32_b200/csrc/ptx.cuh",
-                  "moe_grouped_gemm_fp32_b200/csrc/dg_api.cu"]
+        "dense_large": "TFLOP/s", "contiguous_g4": "TFLOP/s", "masked_g16": "GB/s",
+        "quant_tiny": "GB/s", "quant_tokens_32768": "GB/s", "quant_masked_g16": "GB/s"}
+# the kernel each workload times, and the sources whose hash keys its ncu summary
+KERNEL_SOURCES = {
+    "fp8_gemm_kernel": ["moe_grouped_gemm_fp32_b200/csrc/gemm_kernel.cuh",
+                        "moe_grouped_gemm_fp32_b200/csrc/ptx.cuh",
+                        "moe_grouped_gemm_fp32_b200/csrc/dg_api.cu"],
+    "quant_1x128_kernel": ["moe_grouped_gemm_fp32_b200/csrc/quant_kernel.cuh",
+                           "moe_grouped_gemm_fp32_b200/csrc/quant_api.cu"],
+}
 FLUSH_BYTES = 512 << 20
 
 
-def kernel_source_hash() -> str:
+def is_quant(workload: str) -> bool:
+    return workload.startswith("quant_")
+
+
+def kernel_name(workload: str) -> str:
+    return "quant_1x128_kernel" if is_quant(workload) else "fp8_gemm_kernel"
+
+
+def kernel_source_hash(kernel: str = "fp8_gemm_kernel") -> str:
     h = hashlib.sha256()
-    for f in KERNEL_SOURCES:
+    for f in KERNEL_SOURCES[kernel]:
         with open(os.path.join(ROOT, f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
@@ -61,13 +77,14 @@ def measured_peaks():
 def profiled_traffic(workload: str):
     """DRAM bytes per launch from the committed ncu summary of this workload,
     or None when there is none or the kernel sources changed since."""
-    p = os.path.join(ROOT, "profiles", f"fp8_gemm_kernel_{workload}.md")
+    kernel = kernel_name(workload)
+    p = os.path.join(ROOT, "profiles", f"{kernel}_{workload}.md")
     if not os.path.exists(p):
         return None
     text = open(p).read()
     m = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
     h = re.search(r"kernel_source_hash:\s*([0-9a-f]+)", text)
-    if not m or not h or h.group(1) != kernel_source_hash():
+    if not m or not h or h.group(1) != kernel_source_hash(kernel):
         return None
     return float(m.group(1))
 
@@ -138,6 +155,8 @@ def rank_problem(workload: str, rank: int):
     other ranks the same shapes drawn from another seed (independent
     problems, weak scaling; no data moves between ranks)."""
     import workloads as W
+    if is_quant(workload):
+        return W.make_quant_workload(workload, seed_offset=7919 * rank)
     if rank == 0:
         return W.make_workload(workload)
     spec = dict(W.WORKLOADS[workload])
@@ -163,11 +182,73 @@ def max_over_ranks(values, device, world: int):
 
 
 # ----------------------------------------------------------------------------- our arm
+class GemmCall:
+    """Pinned host inputs, device output and the library call of one GEMM problem."""
+
+    def __init__(self, prob, dev):
+        import numpy as np
+        import torch
+        self.prob = prob
+        self.host = {k: torch.from_numpy(np.ascontiguousarray(v)).pin_memory()
+                     for k, v in (("a", prob.a), ("sfa", prob.sfa), ("b", prob.b), ("sfb", prob.sfb))}
+        if prob.m_indices is not None:
+            self.host["m_indices"] = torch.from_numpy(prob.m_indices).pin_memory()
+        if prob.masked_m is not None:
+            self.host["masked_m"] = torch.from_numpy(prob.masked_m).pin_memory()
+        self.d = torch.empty(prob.d_shape(), dtype=torch.bfloat16, device=dev)
+        self.d_host = torch.empty(prob.d_shape(), dtype=torch.bfloat16).pin_memory()
+
+    def call(self, t, stream):
+        import moe_grouped_gemm_fp32_b200 as dg
+        if self.prob.layout == "dense":
+            dg.dg_fp8_gemm_nt(t["a"], t["sfa"], t["b"][0], t["sfb"][0], self.d, stream)
+        elif self.prob.layout == "contiguous":
+            dg.dg_m_grouped_fp8_gemm_nt_contiguous(t["a"], t["sfa"], t["b"], t["sfb"], self.d,
+                                                   t["m_indices"], stream)
+        else:
+            dg.dg_m_grouped_fp8_gemm_nt_masked(t["a"], t["sfa"], t["b"], t["sfb"], self.d,
+                                               t["masked_m"], stream)
+
+    def read_back(self):
+        self.d_host.copy_(self.d, non_blocking=True)
+
+    def d2h_bytes(self) -> int:
+        return self.d.numel() * self.d.element_size()
+
+
+class QuantCall:
+    """Pinned BF16 activations, device codes and scales, and the quantiser call."""
+
+    def __init__(self, prob, dev):
+        import torch
+        self.prob = prob
+        self.host = {"x": prob.x_bf16().pin_memory()}
+        if prob.masked_m is not None:
+            self.host["masked_m"] = torch.from_numpy(prob.masked_m).pin_memory()
+        shape = tuple(prob.x.shape)
+        sshape = (prob.KB, prob.ld_sfa) if prob.layout == "dense" else (prob.G, prob.KB, prob.ld_sfa)
+        self.q = torch.empty(shape, dtype=torch.uint8, device=dev)
+        self.sfa = torch.empty(sshape, dtype=torch.float32, device=dev)
+        self.q_host = torch.empty(shape, dtype=torch.uint8).pin_memory()
+        self.sfa_host = torch.empty(sshape, dtype=torch.float32).pin_memory()
+
+    def call(self, t, stream):
+        import moe_grouped_gemm_fp32_b200 as dg
+        if self.prob.layout == "dense":
+            dg.dg_per_token_cast_to_fp8(t["x"], self.q, self.sfa, stream)
+        else:
+            dg.dg_per_token_cast_to_fp8_masked(t["x"], self.q, self.sfa, t["masked_m"], stream)
+
+    def read_back(self):
+        self.q_host.copy_(self.q, non_blocking=True)
+        self.sfa_host.copy_(self.sfa, non_blocking=True)
+
+    def d2h_bytes(self) -> int:
+        return self.q.numel() + self.sfa.numel() * 4
+
 def run_ours(args, rank, world, local_rank):
-    import numpy as np
     import torch
     import torch.distributed as dist
-    import workloads as W
     import moe_grouped_gemm_fp32_b200 as dg
     from moe_grouped_gemm_fp32_b200 import build as dg_build
 
@@ -176,15 +257,9 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.set_device(dev)
     prob = rank_problem(args.workload, rank)
 
-    host = {k: torch.from_numpy(np.ascontiguousarray(v)).pin_memory()
-            for k, v in (("a", prob.a), ("sfa", prob.sfa), ("b", prob.b), ("sfb", prob.sfb))}
-    if prob.m_indices is not None:
-        host["m_indices"] = torch.from_numpy(prob.m_indices).pin_memory()
-    if prob.masked_m is not None:
-        host["masked_m"] = torch.from_numpy(prob.masked_m).pin_memory()
+    op = (QuantCall if is_quant(args.workload) else GemmCall)(prob, dev)
+    host = op.host
     devt = {k: v.to(dev, non_blocking=False) for k, v in host.items()}
-    d = torch.empty(prob.d_shape(), dtype=torch.bfloat16, device=dev)
-    d_host = torch.empty(prob.d_shape(), dtype=torch.bfloat16).pin_memory()
     flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     flush_read = torch.ones(FLUSH_BYTES // 8, dtype=torch.float32, device=dev)
 
@@ -196,15 +271,8 @@ def run_ours(args, rank, world, local_rank):
         flush_read.sum()
     stream = torch.cuda.current_stream(dev)
 
-    def call(t, out):
-        if prob.layout == "dense":
-            dg.dg_fp8_gemm_nt(t["a"], t["sfa"], t["b"][0], t["sfb"][0], out, stream)
-        elif prob.layout == "contiguous":
-            dg.dg_m_grouped_fp8_gemm_nt_contiguous(t["a"], t["sfa"], t["b"], t["sfb"], out,
-                                                   t["m_indices"], stream)
-        else:
-            dg.dg_m_grouped_fp8_gemm_nt_masked(t["a"], t["sfa"], t["b"], t["sfb"], out,
-                                               t["masked_m"], stream)
+    def call(t):
+        op.call(t, stream)
 
     def barrier():
         if world > 1:
@@ -215,7 +283,7 @@ def run_ours(args, rank, world, local_rank):
     # ---- device-resident timing
     for i in range(args.warmup):
         flush_l2(i)
-        call(devt, d)
+        call(devt)
     dg.dg_get_device_status(clear=True)
     sampler.start()
     barrier()
@@ -224,7 +292,7 @@ def run_ours(args, rank, world, local_rank):
     for i in range(args.steps):
         flush_l2(i)                      # every step starts from HBM
         starts[i].record(stream)
-        call(devt, d)
+        call(devt)
         ends[i].record(stream)
     barrier()
     clocks = sampler.stop()
@@ -237,8 +305,8 @@ def run_ours(args, rank, world, local_rank):
     # ---- end to end through the public API from pinned host buffers
     for _ in range(max(1, args.warmup // 2)):
         tt = {k: v.to(dev, non_blocking=True) for k, v in host.items()}
-        call(tt, d)
-        d_host.copy_(d, non_blocking=True)
+        call(tt)
+        op.read_back()
     barrier()
     e_start = torch.cuda.Event(enable_timing=True)
     e_end = torch.cuda.Event(enable_timing=True)
@@ -246,13 +314,13 @@ def run_ours(args, rank, world, local_rank):
     e_start.record(stream)
     for _ in range(e2e_steps):
         tt = {k: v.to(dev, non_blocking=True) for k, v in host.items()}
-        call(tt, d)
-        d_host.copy_(d, non_blocking=True)
+        call(tt)
+        op.read_back()
     e_end.record(stream)
     barrier()
     e2e_ms = e_start.elapsed_time(e_end) / e2e_steps
     h2d = sum(v.numel() * v.element_size() for v in host.values())
-    d2h = d.numel() * d.element_size()
+    d2h = op.d2h_bytes()
 
     ms, e2e_ms = max_over_ranks([ms, e2e_ms], dev, world)
     return prob, ms, e2e_ms, h2d, d2h, clocks
@@ -264,12 +332,42 @@ def metric_value(prob, unit, ms, world):
     return prob.flops() * world / (ms * 1e-3) / 1e12
 
 
+def quant_cpu_baseline(prob, budget_s=10.0):
+    """The oracle quantiser as it stands (OpenMP over all host cores) on a
+    bounded sample: evenly spaced valid rows, as many as fit ~budget_s,
+    scaled linearly to the whole workload."""
+    import numpy as np
+    import oracle
+    oracle.build()
+    cores = len(os.sched_getaffinity(0))
+    if prob.layout == "dense":
+        rows = prob.x
+    else:
+        rows = np.concatenate([prob.x[g, :int(prob.masked_m[g])] for g in range(prob.G)])
+    n_all = rows.shape[0]
+    t0 = time.perf_counter()
+    oracle.quantize_1x128(rows[:min(n_all, 16)])
+    per_row = (time.perf_counter() - t0) / max(1, min(n_all, 16))
+    n = int(min(n_all, max(16, budget_s / max(per_row, 1e-9))))
+    pick = rows[:: max(1, n_all // n)][:n]
+    t0 = time.perf_counter()
+    oracle.quantize_1x128(pick)
+    dt = time.perf_counter() - t0
+    secs = dt * n_all / len(pick)
+    value = prob.bytes() / secs / 1e9
+    return {"value": value, "unit": "GB/s", "cores": cores, "kind": "oracle",
+            "sample": f"{len(pick)} of {n_all} valid rows, {dt:.2f} s, scaled linearly to the whole workload",
+            "seconds_per_step": secs}
+
+
 def cpu_baseline(prob, unit, budget_s=10.0):
     """The oracle as it stands (FP64, OpenMP over all host cores) on a bounded
     sample: whole problems repeated until ~budget_s, or a leading slice of the
     output rows when one whole problem would take longer."""
     import numpy as np
     import oracle
+    if not hasattr(prob, "flops"):
+        return quant_cpu_baseline(prob, budget_s)
     oracle.build()
     cores = len(os.sched_getaffinity(0))
     t0 = time.perf_counter()
@@ -336,7 +434,8 @@ def run_reference(args, rank, world):
     value = (prob.bytes() / secs / 1e9) if unit == "GB/s" else (prob.flops() / secs / 1e12)
     line = {"metric": METRIC, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": secs * 1e3, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "scaling": "weak", "vs_baseline": None,
+            "dtype": "f32" if is_quant(args.workload) else "f64", "data": "synthetic",
             "impl": "reference",
             "config": {"workload": args.workload, **shape_config(prob)},
             "cpu_baseline": {"value": value, "unit": unit, "cores": vals[0]["cores"],
@@ -347,6 +446,13 @@ def run_reference(args, rank, world):
 
 
 def shape_config(prob):
+    if not hasattr(prob, "flops"):          # quantiser inputs
+        c = {"layout": prob.layout, "K": prob.K, "in": "bf16", "out": "e4m3 + f32 1x128 scales"}
+        if prob.layout == "dense":
+            c["M"] = prob.M
+        else:
+            c.update(G=prob.G, Mmax=prob.M, valid_rows=prob.valid_rows())
+        return c
     c = {"layout": prob.layout, "N": prob.N, "K": prob.K}
     if prob.layout == "dense":
         c["M"] = prob.M
@@ -404,10 +510,12 @@ def main():
         "metric": METRIC, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": (value / pages[0]) if pages and pages[1] == unit else None,
-        "dtype": "e4m3 (f32 accumulate, bf16 out)", "data": "synthetic",
+        "dtype": ("f32 (bf16 in, e4m3 out)" if is_quant(args.workload)
+                  else "e4m3 (f32 accumulate, bf16 out)"),
+        "data": "synthetic",
         "config": {"workload": args.workload, **shape_config(prob),
                    "l2": "flushed before every step (512 MB write, then 256 MB read)",
-                   "tflops": prob.flops() / (ms * 1e-3) / 1e12,
+                   **({} if is_quant(args.workload) else {"tflops": prob.flops() / (ms * 1e-3) / 1e12}),
                    "gbps": prob.bytes() / (ms * 1e-3) / 1e9},
         "roofline": {"bound": bound, "achieved": achieved, "peak": peak, "unit": runit,
                      "frac": achieved / peak, "traffic": profiled_traffic(args.workload),

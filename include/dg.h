@@ -112,6 +112,43 @@ DG_API dg_status_t dg_m_grouped_fp8_gemm_nt_masked(const uint8_t *a, const float
                                             void *d, const int32_t *masked_m,
                                             int G, int Mmax, int N, int K, void *stream);
 
+/*
+ * Per-token 1x128 activation quantiser (page 2 "技术特性": fine-grained
+ * dynamic scaling; page 3 "核心功能": block-wise scaling): produces the A
+ * operand and sfa of the GEMMs above from BF16 activations.  For each row m
+ * and K-block kb:
+ *   amax = max |x[m, 128kb .. 128kb+127]|
+ *   s    = amax / 448 in FP32 (IEEE division), or 1 when amax == 0
+ *   q[m,k] = E4M3 round-to-nearest-even of clamp(x[m,k] / s, -448, 448),
+ *            with x / s the correctly rounded FP32 quotient
+ *   sfa[kb * ld_sfa + m] = s
+ * The codes are therefore a deterministic function of the inputs, identical
+ * on every run and to any IEEE reference.
+ *   x   [M, K] BF16 row-major (device);  q [M, K] E4M3 (device)
+ *   sfa [KB, ld_sfa] FP32 (device), ld_sfa >= M, ld_sfa % 4 == 0 (so each
+ *       K-block's column starts 16-byte aligned, as the GEMMs' TMA wants);
+ *       entries m >= M are not written.
+ * Inputs must be finite (NaN or infinity gives unspecified codes and scales).
+ * K % 128 == 0; M == 0 is a no-op.  Same pointer, stream and error
+ * conventions as the GEMMs.
+ */
+DG_API dg_status_t dg_per_token_cast_to_fp8(const void *x, uint8_t *q, float *sfa, int ld_sfa,
+                                            int M, int K, void *stream);
+
+/*
+ * The quantiser fused with the masked layout's packing (page 2
+ * "MoE模型专属优化"; page 5 "02", decode): x [G, Mmax, K] BF16, q
+ * [G, Mmax, K] E4M3, sfa [G, KB, ld_sfa] FP32 with ld_sfa >= Mmax -- exactly
+ * the a / sfa operands of dg_m_grouped_fp8_gemm_nt_masked.  Only rows
+ * m < masked_m[g] (device int32 [G]) are read and written; the other rows of
+ * q and sfa are untouched, so the call works unchanged inside a CUDA graph.  A
+ * count outside [0, Mmax] is clamped and recorded as DG_ERR_INVALID_VALUE in
+ * the device status word.  1 <= G <= 1024, G * Mmax < 2^31.
+ */
+DG_API dg_status_t dg_per_token_cast_to_fp8_masked(const void *x, uint8_t *q, float *sfa,
+                                                   int ld_sfa, const int32_t *masked_m, int G,
+                                                   int Mmax, int K, void *stream);
+
 /* Row alignment of the contiguous layout (page 2 "MoE模型专属优化":
  * get_m_alignment_for_contiguous_layout).  Returns 128. */
 DG_API int dg_get_m_alignment_for_contiguous_layout(void);
@@ -139,7 +176,9 @@ DG_API const char *dg_last_cuda_error(void);
  * kernels launched afterwards by this process run with the given debug flags.
  * Flag 1 makes the producer warp issue no loads, so the consumers' bounded
  * waits run out and the kernel records DG_ERR_TIMEOUT in the device status
- * word and returns instead of hanging.  0 restores normal operation.  The
+ * word and returns instead of hanging.  Flag 2 makes the quantisers take the
+ * IEEE division for every element instead of the reciprocal fast path (the
+ * results are identical).  0 restores normal operation.  The
  * wait limit in clock cycles comes from the environment variable
  * DG_WAIT_TIMEOUT_CYCLES, read once (default 2^32). */
 DG_API void dg_debug_set_flags(int flags);

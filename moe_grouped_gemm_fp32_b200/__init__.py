@@ -7,6 +7,7 @@ kernels of ``_dg.so``.  There is no fallback: if the shared library is missing
 or fails to load, importing the library handle raises.
 
 Storage formats (see ``include/dg.h``): A/B are uint8 E4M3 bytes, K-major;
+quantiser inputs are bfloat16 rows;
 sfa is float32 [KB, ld_sfa] ("MN-major"; [G, KB, ld_sfa] for the masked
 layout); sfb is float32 [G, NB, KB]; D is bfloat16.
 """
@@ -57,8 +58,11 @@ def lib() -> ctypes.CDLL:
     L.dg_fp8_gemm_nt.argtypes = [P, P, I, P, P, P, I, I, I, P]
     L.dg_m_grouped_fp8_gemm_nt_contiguous.argtypes = [P, P, I, P, P, P, P, I, I, I, I, P]
     L.dg_m_grouped_fp8_gemm_nt_masked.argtypes = [P, P, I, P, P, P, P, I, I, I, I, P]
+    L.dg_per_token_cast_to_fp8.argtypes = [P, P, P, I, I, I, P]
+    L.dg_per_token_cast_to_fp8_masked.argtypes = [P, P, P, I, P, I, I, I, P]
     for f in ("dg_fp8_gemm_nt", "dg_m_grouped_fp8_gemm_nt_contiguous",
-              "dg_m_grouped_fp8_gemm_nt_masked"):
+              "dg_m_grouped_fp8_gemm_nt_masked", "dg_per_token_cast_to_fp8",
+              "dg_per_token_cast_to_fp8_masked"):
         getattr(L, f).restype = I
     L.dg_get_m_alignment_for_contiguous_layout.argtypes = []
     L.dg_get_m_alignment_for_contiguous_layout.restype = I
@@ -148,6 +152,36 @@ def dg_m_grouped_fp8_gemm_nt_masked(a, sfa, b, sfb, d, masked_m, stream=None):
         G, Mmax, N, K, _stream_handle(stream))
     _check(st, "dg_m_grouped_fp8_gemm_nt_masked")
     return d
+
+
+# --------------------------------------------------------------------------- quantisers
+def dg_per_token_cast_to_fp8(x, q, sfa, stream=None):
+    """Per-token 1x128 quantisation.  x bfloat16 [M,K]; q uint8 [M,K];
+    sfa float32 [KB, ld_sfa] with ld_sfa >= M, a multiple of 4."""
+    import torch
+    M, K = x.shape
+    if tuple(q.shape) != (M, K):
+        raise ValueError("q must have the shape of x")
+    st = lib().dg_per_token_cast_to_fp8(_req(x, torch.bfloat16, "x", 2), _req(q, torch.uint8, "q", 2),
+                                        _req(sfa, torch.float32, "sfa", 2), sfa.shape[-1], M, K,
+                                        _stream_handle(stream))
+    _check(st, "dg_per_token_cast_to_fp8")
+    return q, sfa
+
+
+def dg_per_token_cast_to_fp8_masked(x, q, sfa, masked_m, stream=None):
+    """Quantiser fused with the masked layout.  x bfloat16 [G,Mmax,K]; q uint8
+    [G,Mmax,K]; sfa float32 [G,KB,ld_sfa]; masked_m int32 [G] (device).  Only
+    rows < masked_m[g] are read and written."""
+    import torch
+    G, Mmax, K = x.shape
+    if tuple(q.shape) != (G, Mmax, K):
+        raise ValueError("q must have the shape of x")
+    st = lib().dg_per_token_cast_to_fp8_masked(
+        _req(x, torch.bfloat16, "x", 3), _req(q, torch.uint8, "q", 3), _req(sfa, torch.float32, "sfa", 3),
+        sfa.shape[-1], _req(masked_m, torch.int32, "masked_m", 1), G, Mmax, K, _stream_handle(stream))
+    _check(st, "dg_per_token_cast_to_fp8_masked")
+    return q, sfa
 
 
 # --------------------------------------------------------------------------- helpers

@@ -11,13 +11,16 @@
 #include <mutex>
 
 #include "dg.h"
+#include "api_common.h"
 #include "gemm_kernel.cuh"
 
 namespace {
-
 __device__ unsigned g_dg_status = 0u;
-
 thread_local char t_last_cuda_error[256] = "";
+int g_debug_flags = 0;
+}  // namespace
+
+namespace dg_host {
 
 dg_status_t cuda_fail(cudaError_t e, const char *what) {
     std::snprintf(t_last_cuda_error, sizeof(t_last_cuda_error), "%s: %s", what,
@@ -25,18 +28,21 @@ dg_status_t cuda_fail(cudaError_t e, const char *what) {
     return DG_ERR_CUDA;
 }
 
+int debug_flags() { return g_debug_flags; }
+
+bool verbose() {
+    static bool v = [] {
+        const char *s = std::getenv("DG_VERBOSE");
+        return s && s[0] == '1';
+    }();
+    return v;
+}
+
 // ------------------------------------------------------------------ device info
-constexpr int kMaxDevices = 64;
-
-struct DeviceInfo {
-    bool ready = false;
-    bool supported = false;
-    int num_sms = 0;
-    unsigned *status = nullptr;   // device address of g_dg_status
-};
-
+namespace {
 DeviceInfo g_devices[kMaxDevices];
 std::mutex g_mutex;
+}  // namespace
 
 dg_status_t device_info(const DeviceInfo **out) {
     int dev = 0;
@@ -68,6 +74,11 @@ dg_status_t device_info(const DeviceInfo **out) {
     *out = &info;
     return DG_SUCCESS;
 }
+
+}  // namespace dg_host
+
+namespace {
+using namespace dg_host;
 
 // ------------------------------------------------------------------ tensor maps
 using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
@@ -118,8 +129,6 @@ dg_status_t make_map(CUtensorMap *m, const void *base, long long K, long long ro
 }
 
 // ------------------------------------------------------------------ validation
-bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
-
 dg_status_t check_common(const void *a, const float *sfa, int ld_sfa, const void *b,
                          const float *sfb, const void *d, int rows, int N, int K) {
     if (!a || !sfa || !b || !sfb || !d) return DG_ERR_INVALID_VALUE;
@@ -139,17 +148,6 @@ long long timeout_cycles() {
         const char *s = std::getenv("DG_WAIT_TIMEOUT_CYCLES");
         long long x = s ? std::atoll(s) : 0;
         return x > 0 ? x : (1LL << 32);   // ~2 s at 2 GHz; legitimate waits are micro- to milliseconds
-    }();
-    return v;
-}
-
-int g_debug_flags = 0;
-
-// DG_VERBOSE=1 prints each launch's configuration to stderr.
-bool verbose() {
-    static bool v = [] {
-        const char *s = std::getenv("DG_VERBOSE");
-        return s && s[0] == '1';
     }();
     return v;
 }
@@ -291,6 +289,7 @@ dg::Params base_params(const float *sfa, int ld_sfa, const float *sfb, void *d, 
     p.debug_flags = g_debug_flags;
     return p;
 }
+
 
 
 }  // namespace
@@ -488,7 +487,9 @@ const char *dg_last_cuda_error(void) { return t_last_cuda_error; }
 // Test hook (not part of the GEMM contract): kernels launched afterwards on
 // this process run with the given debug flags.  Flag 1 makes the producer warp
 // issue no loads, so the consumers' bounded waits run out and the kernel
-// reports DG_ERR_TIMEOUT through the status word instead of hanging.
+// reports DG_ERR_TIMEOUT through the status word instead of hanging.  Flag 2
+// makes the quantiser take the IEEE division for every element (its results
+// are identical; tests compare the two paths).
 void dg_debug_set_flags(int flags) { g_debug_flags = flags; }
 
 }  // extern "C"

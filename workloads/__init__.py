@@ -277,3 +277,105 @@ def make_workload(name: str) -> Problem:
     if kind == "contiguous":
         return make_contiguous_multinomial(w["G"], w["tokens"], w["N"], w["K"], w["seed"], name=name)
     return make_masked_uniform(w["G"], w["Mmax"], w["N"], w["K"], w["seed"], name=name)
+
+
+# ----------------------------------------------------------------------------- quantiser inputs
+@dataclasses.dataclass
+class QuantProblem:
+    """Inputs of the per-token 1x128 quantiser: BF16 activations, held here as
+    their exact float32 values.  Dense: x [M, K]; masked: x [G, Mmax, K] with
+    valid rows m < masked_m[g] (the other rows hold NaN, which the quantiser
+    must never read)."""
+    layout: str
+    x: np.ndarray
+    masked_m: Optional[np.ndarray] = None
+    name: str = ""
+
+    @property
+    def K(self) -> int:
+        return int(self.x.shape[-1])
+
+    @property
+    def KB(self) -> int:
+        return self.K // BLOCK
+
+    @property
+    def G(self) -> int:
+        return 1 if self.layout == "dense" else int(self.x.shape[0])
+
+    @property
+    def M(self) -> int:
+        """Rows per group (dense: M; masked: Mmax)."""
+        return int(self.x.shape[-2])
+
+    @property
+    def ld_sfa(self) -> int:
+        return tma_aligned(max(self.M, 1))
+
+    def valid_rows(self) -> int:
+        return self.M if self.layout == "dense" else int(self.masked_m.sum())
+
+    def bytes(self) -> float:
+        """Algorithmic bytes: BF16 in, E4M3 out, one FP32 scale per 128 out."""
+        return float(self.valid_rows()) * (2 * self.K + self.K + 4 * self.KB)
+
+    def x_bf16(self) -> torch.Tensor:
+        return torch.from_numpy(np.ascontiguousarray(self.x)).to(torch.bfloat16)
+
+
+def _bf16_exact(x32: np.ndarray) -> np.ndarray:
+    return torch.from_numpy(x32).to(torch.bfloat16).to(torch.float32).numpy()
+
+
+def _activations(rng, rows: int, K: int, outliers: bool) -> np.ndarray:
+    x = _normal(rng, (rows, K))
+    if outliers:
+        cols = rng.choice(K, size=K // 100, replace=False)
+        x[:, cols] *= 20.0
+    return _bf16_exact(x)
+
+
+def make_activations(M: int, K: int, seed: int, outliers: bool = True, name: str = "") -> QuantProblem:
+    """Dense activations x [M, K]: N(0,1), one fixed set of floor(0.01*K)
+    outlier columns x20 (as the GEMM workloads' A), rounded to BF16."""
+    rng = np.random.default_rng(seed)
+    return QuantProblem("dense", _activations(rng, M, K, outliers), name=name)
+
+
+def make_activations_masked(masked_m, Mmax: int, K: int, seed: int, outliers: bool = True,
+                            name: str = "", poison: bool = True) -> QuantProblem:
+    """Masked activations x [G, Mmax, K]; rows >= masked_m[g] are NaN."""
+    rng = np.random.default_rng(seed)
+    masked_m = np.asarray(masked_m, dtype=np.int32)
+    G = len(masked_m)
+    x = _activations(rng, G * Mmax, K, outliers).reshape(G, Mmax, K)
+    if poison:
+        for g in range(G):
+            x[g, masked_m[g]:] = np.nan
+    return QuantProblem("masked", x, masked_m=masked_m, name=name)
+
+
+def make_activations_masked_uniform(G: int, Mmax: int, K: int, seed: int,
+                                    name: str = "") -> QuantProblem:
+    """masked_m[g] ~ Uniform{0..Mmax} from ``seed``; values from seed+1000."""
+    rng = np.random.default_rng(seed)
+    masked_m = rng.integers(0, Mmax + 1, size=G).astype(np.int32)
+    return make_activations_masked(masked_m, Mmax, K, seed + 1000, name=name)
+
+
+# Quantiser workloads: the activations that feed the contiguous prefill GEMM
+# (32768 tokens, K = 7168) and the masked decode GEMM (16 groups, Mmax 256).
+QUANT_WORKLOADS = {
+    "quant_tiny": dict(kind="dense", M=130, K=640, seed=8),
+    "quant_tokens_32768": dict(kind="dense", M=32768, K=7168, seed=6),
+    "quant_masked_g16": dict(kind="masked", G=16, Mmax=256, K=7168, seed=7),
+}
+
+
+def make_quant_workload(name: str, seed_offset: int = 0) -> QuantProblem:
+    w = dict(QUANT_WORKLOADS[name])
+    kind = w.pop("kind")
+    seed = w.pop("seed") + seed_offset
+    if kind == "dense":
+        return make_activations(w["M"], w["K"], seed, name=name)
+    return make_activations_masked_uniform(w["G"], w["Mmax"], w["K"], seed, name=name)
