@@ -1,4 +1,5 @@
-"""CPU oracle for the FP8 block-scaled NT GEMM (dense / contiguous / masked).
+"""CPU oracle for the FP8 block-scaled NT GEMM (dense / contiguous / masked /
+K-grouped) and the per-token 1x128 activation quantiser.
 
 TEST INFRASTRUCTURE ONLY: imported by ``tests/``, ``__graft_entry__.smoke()``
 and the CPU-baseline leg of ``bench.py``; never by the library.  It shares no
@@ -9,6 +10,12 @@ definition for tiny shapes.
 
 Definition (DeepGEMM pages, page 2 "技术特性" and page 3 "核心功能"):
     D[m,n] = sum_kb sA[m,kb] * sB[n//128,kb] * sum_{k in kb} A[m,k] * B[n,k]
+K-grouped (page 3 "核心功能", k_grouped_gemm): group g sums only over its own
+ks[g] consecutive K columns, D[g] = the same sum over those K-blocks.
+Quantiser (page 2 "技术特性", dynamic fine-grained scaling): per row and
+128-wide K-block, s = amax / 448 in FP32, q = E4M3_RNE(clamp(x / s, +-448)).
+Every function is pinned (tests/test_oracle.py, tests/test_oracle_quant.py,
+tests/test_oracle_mutants.py); none is "parity unpinned".
 """
 from __future__ import annotations
 
@@ -55,6 +62,10 @@ def _load():
         for f in ("oracle_fp8_gemm_nt", "oracle_m_grouped_contiguous",
                   "oracle_m_grouped_masked", "oracle_points"):
             getattr(lib, f).restype = ctypes.c_int
+        lib.oracle_k_grouped.argtypes = [P, P, L, P, P, P, L, L, L, L, P]
+        lib.oracle_k_grouped.restype = ctypes.c_int
+        lib.oracle_k_grouped_points.argtypes = [P, P, L, P, P, P, L, L, L, L, L, P, P, P, P]
+        lib.oracle_k_grouped_points.restype = ctypes.c_int
         lib.oracle_e4m3_encode.argtypes = [ctypes.c_float]
         lib.oracle_e4m3_encode.restype = ctypes.c_uint8
         lib.oracle_quantize_1x128.argtypes = [P, L, L, P, P, L]
@@ -117,11 +128,37 @@ def gemm_masked(a, sfa, ld_sfa, b, sfb, masked_m, G, Mmax, N, K,
     return d
 
 
+def gemm_k_grouped(a, sfa, ld_sfa, b, sfb, ks, M, N, K) -> np.ndarray:
+    """K-grouped: group g reduces over its ks[g] K columns only; returns
+    float64 [G, M, N] (zeros for an empty group)."""
+    a, b = _c(a, np.uint8), _c(b, np.uint8)
+    sfa, sfb = _c(sfa, np.float32), _c(sfb, np.float32)
+    ks = _c(ks, np.int32)
+    G = len(ks)
+    d = np.empty((G, M, N), dtype=np.float64)
+    rc = _load().oracle_k_grouped(_p(a), _p(sfa), ld_sfa, _p(b), _p(sfb), _p(ks), G, M, N, K, _p(d))
+    if rc:
+        raise ValueError(f"oracle_k_grouped rejected the input (rc={rc})")
+    return d
+
+
 _LAYOUT_CODE = {"dense": 0, "contiguous": 1, "masked": 2}
 
 
 def points(prob, grp, row, col) -> np.ndarray:
     """Sampled outputs D[grp, row, col] of a ``workloads.Problem``."""
+    if prob.layout == "k_grouped":
+        a, b = _c(prob.a, np.uint8), _c(prob.b[0], np.uint8)
+        sfa, sfb = _c(prob.sfa, np.float32), _c(prob.sfb[0], np.float32)
+        ks = _c(prob.ks, np.int32)
+        grp, row, col = (_c(x, np.int32) for x in (grp, row, col))
+        out = np.empty(len(row), dtype=np.float64)
+        rc = _load().oracle_k_grouped_points(_p(a), _p(sfa), prob.ld_sfa, _p(b), _p(sfb), _p(ks),
+                                             len(ks), prob.M, prob.N, prob.K, len(row),
+                                             _p(grp), _p(row), _p(col), _p(out))
+        if rc:
+            raise ValueError(f"oracle_k_grouped_points rejected the input (rc={rc})")
+        return out
     a, b = _c(prob.a, np.uint8), _c(prob.b, np.uint8)
     sfa, sfb = _c(prob.sfa, np.float32), _c(prob.sfb, np.float32)
     mi = None if prob.m_indices is None else _c(prob.m_indices, np.int32)
@@ -144,6 +181,9 @@ def solve(prob) -> np.ndarray:
     if prob.layout == "contiguous":
         return gemm_contiguous(prob.a, prob.sfa, prob.ld_sfa, prob.b, prob.sfb,
                                prob.m_indices, prob.M, prob.N, prob.K, prob.G)
+    if prob.layout == "k_grouped":
+        return gemm_k_grouped(prob.a, prob.sfa, prob.ld_sfa, prob.b[0], prob.sfb[0], prob.ks,
+                              prob.M, prob.N, prob.K)
     return gemm_masked(prob.a, prob.sfa, prob.ld_sfa, prob.b, prob.sfb, prob.masked_m,
                        prob.G, prob.M, prob.N, prob.K)
 

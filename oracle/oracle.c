@@ -38,7 +38,9 @@
  * and closed-form values; brute force on tiny shapes; the all-ones-scale case
  * against a float64 matmul; exact integer cases with power-of-two scales
  * against exact integer arithmetic; identity and zero operands; scale
- * linearity; grouped == per-group dense.
+ * linearity; grouped == per-group dense; K-grouped: the groups' outputs sum
+ * to the dense GEMM over all of K (exactly, for integer cases), one group ==
+ * dense, an empty group gives zeros, brute force on tiny shapes.
  */
 #include <math.h>
 #include <stdint.h>
@@ -200,6 +202,84 @@ int oracle_points(int layout, const uint8_t *a, const float *sfa, long ld_sfa,
         }
         out[i] = block_scaled_dot(arow, sa, ld_sfa, b + (g * N + n) * K,
                                   sfb + (g * NB + n / ORC_BLOCK) * KB, K, lut);
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------------------------
+ * K-grouped GEMM (DeepGEMM page 3 "核心功能": the k_grouped_gemm family next to
+ * the m-grouped one -- groups laid out along K, the weight-gradient shape of
+ * MoE training, where the reduced dimension is each expert's tokens).
+ *
+ * Group g owns ks[g] consecutive K columns (ks[g] % 128 == 0, sum = K), i.e.
+ * the K-blocks [o_g, o_g + ks[g]/128) with o_g the exclusive prefix of
+ * ks/128, of both A [M,K] and B [N,K] and of their scales (the dense layout's
+ * sfa [KB][ld_sfa] and sfb [NB][KB]).  Each group has its own output:
+ *
+ *   D[g][m][n] = sum_{kb in group g} sA[m,kb] * sB[n/128,kb] * (A_blk . B_blk)
+ *
+ * -- the dense definition restricted to the group's K-blocks; an empty group
+ * gives zeros.
+ * ------------------------------------------------------------------------ */
+static int check_ks(const int32_t *ks, long G, long K)
+{
+    long sum = 0;
+    for (long g = 0; g < G; ++g) {
+        if (ks[g] < 0 || ks[g] % ORC_BLOCK != 0) return 2;
+        sum += ks[g];
+    }
+    return sum == K ? 0 : 2;
+}
+
+int oracle_k_grouped(const uint8_t *a, const float *sfa, long ld_sfa,
+                     const uint8_t *b, const float *sfb, const int32_t *ks,
+                     long G, long M, long N, long K, double *d)
+{
+    if (check_shape(M, N, K) || G <= 0) return 1;
+    if (check_ks(ks, G, K)) return 2;
+    double lut[256];
+    oracle_e4m3_table(lut);
+    long KB = K / ORC_BLOCK;
+    long off = 0;
+    for (long g = 0; g < G; ++g) {
+        const long kb0 = off / ORC_BLOCK, Kg = ks[g];
+        #pragma omp parallel for schedule(dynamic, 1)
+        for (long m = 0; m < M; ++m)
+            for (long n = 0; n < N; ++n)
+                d[(g * M + m) * N + n] =
+                    Kg == 0 ? 0.0
+                            : block_scaled_dot(a + m * K + kb0 * ORC_BLOCK, sfa + kb0 * ld_sfa + m, ld_sfa,
+                                               b + n * K + kb0 * ORC_BLOCK,
+                                               sfb + (n / ORC_BLOCK) * KB + kb0, Kg, lut);
+        off += Kg;
+    }
+    return 0;
+}
+
+/* Sampled outputs D[grp[i]][row[i]][col[i]] of the K-grouped GEMM. */
+int oracle_k_grouped_points(const uint8_t *a, const float *sfa, long ld_sfa,
+                            const uint8_t *b, const float *sfb, const int32_t *ks,
+                            long G, long M, long N, long K, long npts,
+                            const int32_t *grp, const int32_t *row, const int32_t *col,
+                            double *out)
+{
+    if (check_shape(M, N, K) || G <= 0) return 1;
+    if (check_ks(ks, G, K)) return 2;
+    for (long i = 0; i < npts; ++i)
+        if (grp[i] < 0 || grp[i] >= G || row[i] < 0 || row[i] >= M || col[i] < 0 || col[i] >= N)
+            return 3;
+    double lut[256];
+    oracle_e4m3_table(lut);
+    long KB = K / ORC_BLOCK;
+    #pragma omp parallel for schedule(dynamic, 1)
+    for (long i = 0; i < npts; ++i) {
+        long g = grp[i], m = row[i], n = col[i], off = 0;
+        for (long h = 0; h < g; ++h) off += ks[h];
+        const long kb0 = off / ORC_BLOCK, Kg = ks[g];
+        out[i] = Kg == 0 ? 0.0
+                         : block_scaled_dot(a + m * K + kb0 * ORC_BLOCK, sfa + kb0 * ld_sfa + m, ld_sfa,
+                                            b + n * K + kb0 * ORC_BLOCK,
+                                            sfb + (n / ORC_BLOCK) * KB + kb0, Kg, lut);
     }
     return 0;
 }

@@ -213,3 +213,55 @@ def test_oracle_rejects_bad_shapes(oracle_lib):
     with pytest.raises(ValueError):
         oracle_lib.gemm_dense(np.zeros((2, 100), np.uint8), np.zeros((1, 4), np.float32), 4,
                               np.zeros((2, 100), np.uint8), np.zeros((1, 1), np.float32), 2, 2, 100)
+
+
+# --------------------------------------------------------------------------- k-grouped
+def test_k_grouped_brute_force(oracle_lib):
+    """Each group equals the exact brute force over its own K columns (a
+    second statement of the definition, with the K slicing done here)."""
+    rng = np.random.default_rng(301)
+    M, N, ks = 3, 130, np.array([128, 0, 256], np.int32)
+    K = int(ks.sum())
+    a, b = _rand_bytes(rng, (M, K)), _rand_bytes(rng, (N, K))
+    KB, NB = K // 128, (N + 127) // 128
+    sa = rng.uniform(0.01, 2.0, size=(M, KB)).astype(np.float32)
+    sb = rng.uniform(0.01, 2.0, size=(NB, KB)).astype(np.float32)
+    d = oracle_lib.gemm_k_grouped(a, W.sfa_mn_major(sa), W.tma_aligned(M), b, sb, ks, M, N, K)
+    off = 0
+    for g, kg in enumerate(ks):
+        c0, c1, b0, b1 = off, off + kg, off // 128, (off + kg) // 128
+        if kg == 0:
+            assert (d[g] == 0).all()
+        else:
+            ref = brute.gemm(a[:, c0:c1], sa[:, b0:b1], b[:, c0:c1], sb[:, b0:b1], M, N, int(kg))
+            for m in range(M):
+                for n in range(N):
+                    assert abs(d[g, m, n] - float(ref[m][n])) <= 1e-13 * max(1.0, abs(float(ref[m][n])))
+        off += kg
+
+
+def test_k_grouped_sums_to_dense_exactly(oracle_lib):
+    """Linearity over K: the groups' outputs add up to the dense GEMM over all
+    of K -- exactly, with integer operands and power-of-two scales."""
+    M, N, K = 6, 136, 768
+    a, sa, b, sb, exact = _exact_case(23, M, N, K)
+    ks = np.array([256, 128, 0, 384], np.int32)
+    d = oracle_lib.gemm_k_grouped(a, W.sfa_mn_major(sa), W.tma_aligned(M), b, sb, ks, M, N, K)
+    assert d.shape == (4, M, N)
+    assert np.array_equal(d.sum(axis=0), exact)
+    assert (d[2] == 0).all()
+    one = oracle_lib.gemm_k_grouped(a, W.sfa_mn_major(sa), W.tma_aligned(M), b, sb,
+                                    np.array([K], np.int32), M, N, K)
+    assert np.array_equal(one[0], oracle_lib.gemm_dense(a, W.sfa_mn_major(sa), W.tma_aligned(M), b, sb, M, N, K))
+
+
+def test_k_grouped_points_and_rejections(oracle_lib):
+    p = W.make_k_grouped([256, 128, 384], 40, 200, seed=5)
+    full = oracle_lib.solve(p)
+    rng = np.random.default_rng(0)
+    g, r, c = rng.integers(0, 3, 50), rng.integers(0, 40, 50), rng.integers(0, 200, 50)
+    assert np.array_equal(oracle_lib.points(p, g, r, c), full[g, r, c])
+    with pytest.raises(ValueError):      # group sizes must be multiples of 128
+        oracle_lib.gemm_k_grouped(p.a, p.sfa, p.ld_sfa, p.b[0], p.sfb[0], [200, 184, 384], 40, 200, 768)
+    with pytest.raises(ValueError):      # and add up to K
+        oracle_lib.gemm_k_grouped(p.a, p.sfa, p.ld_sfa, p.b[0], p.sfb[0], [256, 128, 256], 40, 200, 768)

@@ -27,6 +27,15 @@ MUTANTS = {
         ("p += lut[ak[i]] * lut[bk[i]];", "p += lut[ak[i]] * lut[bk[(i + 1) % ORC_BLOCK]];"),
     "weight scale ignored":
         ("((double)sa[kb * sa_stride] * (double)sb[kb]) * p", "((double)sa[kb * sa_stride]) * p"),
+    "k-grouped: every group starts at K-block 0":
+        ("        off += Kg;\n", "        off += 0;\n"),
+    "k-grouped: group's activation scales taken from K-block 0":
+        ("sfa + kb0 * ld_sfa + m", "sfa + m"),
+    "quantiser: scale amax / 240 (the E4M3 'fnuz' maximum)":
+        ("float s = amax / 448.0f;", "float s = amax / 240.0f;"),
+    "quantiser: encoder rounds ties away from zero":
+        ("if (frac > 0.5 || (frac == 0.5 && fmod(lo, 2.0) != 0.0)) r = lo + 1.0;",
+         "if (frac >= 0.5) r = lo + 1.0;"),
 }
 
 
@@ -42,6 +51,7 @@ def test_pins_catch_mutant(name, tmp_path):
                            "-o", str(so), str(mutated), "-lm"])
     env = dict(os.environ, ORACLE_SO=str(so))
     r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
-                        os.path.join(ROOT, "tests", "test_oracle.py")],
+                        os.path.join(ROOT, "tests", "test_oracle.py"),
+                        os.path.join(ROOT, "tests", "test_oracle_quant.py")],
                        cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
     assert r.returncode != 0, f"pins did not catch: {name}\n{r.stdout[-2000:]}"

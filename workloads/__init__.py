@@ -95,8 +95,8 @@ def sfa_mn_major(s_rows: np.ndarray, ld: Optional[int] = None) -> np.ndarray:
 @dataclasses.dataclass
 class Problem:
     """One GEMM problem in the library's storage formats (host numpy arrays)."""
-    layout: str                    # "dense" | "contiguous" | "masked"
-    M: int                         # dense: rows; contiguous: M_total; masked: Mmax
+    layout: str                    # "dense" | "contiguous" | "masked" | "k_grouped"
+    M: int                         # dense, k_grouped: rows; contiguous: M_total; masked: Mmax
     N: int
     K: int
     G: int
@@ -108,6 +108,7 @@ class Problem:
     m_indices: Optional[np.ndarray] = None   # int32 [M_total] (contiguous)
     masked_m: Optional[np.ndarray] = None    # int32 [G] (masked)
     name: str = ""
+    ks: Optional[np.ndarray] = None          # int32 [G] (k_grouped: K columns per group)
 
     @property
     def KB(self) -> int:
@@ -118,14 +119,14 @@ class Problem:
         return (self.N + BLOCK - 1) // BLOCK
 
     def valid_rows(self) -> int:
-        if self.layout == "dense":
+        if self.layout in ("dense", "k_grouped"):
             return self.M
         if self.layout == "contiguous":
             return int((self.m_indices >= 0).sum())
         return int(self.masked_m.sum())
 
     def groups_touched(self) -> int:
-        if self.layout == "dense":
+        if self.layout in ("dense", "k_grouped"):
             return 1
         if self.layout == "contiguous":
             return int(len(np.unique(self.m_indices[self.m_indices >= 0])))
@@ -136,13 +137,17 @@ class Problem:
         return 2.0 * self.valid_rows() * self.N * self.K
 
     def bytes(self) -> float:
-        """Algorithmic bytes: A + B + sA + sB + D over valid rows / touched groups."""
+        """Algorithmic bytes: A + B + sA + sB + D over valid rows / touched groups
+        (k_grouped: A, B and their scales once, one D per group)."""
         rows, g = self.valid_rows(), self.groups_touched()
+        if self.layout == "k_grouped":
+            return float(rows * self.K + self.N * self.K + rows * self.KB * 4
+                         + self.NB * self.KB * 4 + self.G * rows * self.N * 2)
         return float(rows * self.K + g * self.N * self.K + rows * self.KB * 4
                      + g * self.NB * self.KB * 4 + rows * self.N * 2)
 
     def d_shape(self):
-        if self.layout == "masked":
+        if self.layout in ("masked", "k_grouped"):
             return (self.G, self.M, self.N)
         return (self.M, self.N)
 
@@ -257,6 +262,30 @@ def make_masked_uniform(G: int, Mmax: int, N: int, K: int, seed: int,
     return make_masked(masked_m, Mmax, N, K, seed + 1000, name=name)
 
 
+def make_k_grouped(ks, M: int, N: int, seed: int, name: str = "", outliers: bool = False) -> Problem:
+    """K-grouped problem: group g owns ks[g] consecutive K columns (multiples
+    of 128) of A [M, K] and B [N, K], K = sum(ks); D is [G, M, N].  A and B ~
+    N(0,1), quantised like the dense layout (1x128 rows of A, 128x128 blocks
+    of B), so each group's K-blocks carry their own scales."""
+    ks = np.asarray(ks, dtype=np.int32)
+    K = int(ks.sum())
+    assert K > 0 and (ks % BLOCK == 0).all() and (ks >= 0).all()
+    p = make_dense(M, N, K, seed, outliers=outliers, name=name)
+    return Problem("k_grouped", M, N, K, len(ks), p.a, p.sfa, p.ld_sfa, p.b, p.sfb,
+                   name=name, ks=ks)
+
+
+def make_k_grouped_multinomial(G: int, tokens: int, M: int, N: int, seed: int,
+                               name: str = "") -> Problem:
+    """Tokens per expert from multinomial(tokens, [1/G]*G) drawn from ``seed``,
+    each rounded up to a multiple of 128 (the K alignment); operands from
+    seed+1000."""
+    rng = np.random.default_rng(seed)
+    counts = rng.multinomial(tokens, [1.0 / G] * G)
+    ks = ((counts + BLOCK - 1) // BLOCK * BLOCK).astype(np.int32)
+    return make_k_grouped(ks, M, N, seed + 1000, name=name)
+
+
 # The five workloads of the method's benchmark set (shapes from the pages'
 # benchmark table, DeepGEMM page 2 "性能实测", plus the expert counts).
 WORKLOADS = {
@@ -266,6 +295,8 @@ WORKLOADS = {
     "dense_large": dict(kind="dense", M=4096, N=7168, K=16384, seed=3),
     "contiguous_g4": dict(kind="contiguous", G=4, tokens=32768, N=4096, K=7168, seed=4),
     "masked_g16": dict(kind="masked", G=16, Mmax=256, N=4096, K=7168, seed=5),
+    # weight-gradient shape of MoE training: 4 experts, 32768 tokens along K
+    "kgrouped_g4": dict(kind="k_grouped", G=4, tokens=32768, M=4096, N=7168, seed=9),
 }
 
 
@@ -276,6 +307,8 @@ def make_workload(name: str) -> Problem:
         return make_dense(name=name, **w)
     if kind == "contiguous":
         return make_contiguous_multinomial(w["G"], w["tokens"], w["N"], w["K"], w["seed"], name=name)
+    if kind == "k_grouped":
+        return make_k_grouped_multinomial(w["G"], w["tokens"], w["M"], w["N"], w["seed"], name=name)
     return make_masked_uniform(w["G"], w["Mmax"], w["N"], w["K"], w["seed"], name=name)
 
 
