@@ -38,6 +38,7 @@ DEFAULT_WORKLOAD = "dense_decode_m64"
 PAGES_NUMBER = {"dense_decode_m64": (1688.0, "GB/s")}
 UNIT = {"dense_tiny": "TFLOP/s", "dense_decode_m64": "GB/s", "dense_decode_m128": "GB/s",
         "dense_large": "TFLOP/s", "contiguous_g4": "TFLOP/s", "masked_g16": "GB/s",
+        "kgrouped_g4": "TFLOP/s",
         "quant_tiny": "GB/s", "quant_tokens_32768": "GB/s", "quant_masked_g16": "GB/s"}
 # the kernel each workload times, and the sources whose hash keys its ncu summary
 KERNEL_SOURCES = {
@@ -166,6 +167,8 @@ def rank_problem(workload: str, rank: int):
         return W.make_dense(**spec)
     if kind == "contiguous":
         return W.make_contiguous_multinomial(spec["G"], spec["tokens"], spec["N"], spec["K"], spec["seed"])
+    if kind == "k_grouped":
+        return W.make_k_grouped_multinomial(spec["G"], spec["tokens"], spec["M"], spec["N"], spec["seed"])
     return W.make_masked_uniform(spec["G"], spec["Mmax"], spec["N"], spec["K"], spec["seed"])
 
 
@@ -195,6 +198,8 @@ class GemmCall:
             self.host["m_indices"] = torch.from_numpy(prob.m_indices).pin_memory()
         if prob.masked_m is not None:
             self.host["masked_m"] = torch.from_numpy(prob.masked_m).pin_memory()
+        if prob.ks is not None:
+            self.host["ks"] = torch.from_numpy(prob.ks).pin_memory()
         self.d = torch.empty(prob.d_shape(), dtype=torch.bfloat16, device=dev)
         self.d_host = torch.empty(prob.d_shape(), dtype=torch.bfloat16).pin_memory()
 
@@ -205,6 +210,9 @@ class GemmCall:
         elif self.prob.layout == "contiguous":
             dg.dg_m_grouped_fp8_gemm_nt_contiguous(t["a"], t["sfa"], t["b"], t["sfb"], self.d,
                                                    t["m_indices"], stream)
+        elif self.prob.layout == "k_grouped":
+            dg.dg_k_grouped_fp8_gemm_nt_contiguous(t["a"], t["sfa"], t["b"][0], t["sfb"][0], self.d,
+                                                   t["ks"], stream)
         else:
             dg.dg_m_grouped_fp8_gemm_nt_masked(t["a"], t["sfa"], t["b"], t["sfb"], self.d,
                                                t["masked_m"], stream)
@@ -372,6 +380,25 @@ def cpu_baseline(prob, unit, budget_s=10.0):
     cores = len(os.sched_getaffinity(0))
     t0 = time.perf_counter()
     probe_rows = max(1, min(prob.M, 8))
+    if prob.layout == "k_grouped":
+        # output rows are (group, row) pairs: G * M of them, each of N columns
+        sel = [(g, m) for g in range(prob.G) for m in range(prob.M)]
+        t0 = time.perf_counter()
+        probe = sel[:: max(1, len(sel) // probe_rows)][:probe_rows]
+        oracle.points(prob, np.repeat([q[0] for q in probe], prob.N), np.repeat([q[1] for q in probe], prob.N),
+                      np.tile(np.arange(prob.N), len(probe)))
+        per_row = (time.perf_counter() - t0) / len(probe)
+        n_rows = max(1, min(len(sel), int(budget_s / per_row)))
+        pick = sel[:: max(1, len(sel) // n_rows)][:n_rows]
+        t0 = time.perf_counter()
+        oracle.points(prob, np.repeat([q[0] for q in pick], prob.N), np.repeat([q[1] for q in pick], prob.N),
+                      np.tile(np.arange(prob.N), len(pick)))
+        dt = time.perf_counter() - t0
+        secs = dt * len(sel) / len(pick)
+        value = (prob.bytes() / secs / 1e9) if unit == "GB/s" else (prob.flops() / secs / 1e12)
+        return {"value": value, "unit": unit, "cores": cores, "kind": "oracle",
+                "sample": f"{len(pick)} of {len(sel)} (group, row) output rows (all N columns), {dt:.1f} s, "
+                          f"scaled linearly to the whole workload", "seconds_per_step": secs}
     if prob.layout == "masked":
         g = int(np.argmax(prob.masked_m))
         rows = np.arange(min(probe_rows, int(prob.masked_m[g])))
@@ -458,6 +485,8 @@ def shape_config(prob):
         c["M"] = prob.M
     elif prob.layout == "contiguous":
         c.update(G=prob.G, M_total=prob.M, valid_rows=prob.valid_rows())
+    elif prob.layout == "k_grouped":
+        c.update(G=prob.G, M=prob.M, ks=[int(k) for k in prob.ks])
     else:
         c.update(G=prob.G, Mmax=prob.M, valid_rows=prob.valid_rows())
     return c

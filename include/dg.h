@@ -113,6 +113,29 @@ DG_API dg_status_t dg_m_grouped_fp8_gemm_nt_masked(const uint8_t *a, const float
                                             int G, int Mmax, int N, int K, void *stream);
 
 /*
+ * K-grouped GEMM, groups contiguous along K (page 3 "核心功能": the
+ * k_grouped_gemm family -- the weight-gradient shape of MoE training, where
+ * the reduced dimension is each expert's tokens).  Group g owns ks[g]
+ * consecutive K columns of A and B (and the matching K-blocks of sfa / sfb);
+ * its output is the block-scaled sum over those K-blocks only:
+ *   D[g][m][n] = sum_{kb in group g} sA[m,kb] * sB[n/128,kb] * (A_kb . B_kb)
+ *   a   [M, K] E4M3;  sfa [KB, ld_sfa] FP32, ld_sfa >= M   (dense layout)
+ *   b   [N, K] E4M3;  sfb [NB, KB] FP32                     (dense layout)
+ *   d   [G, M, N] BF16, fully written (zeros for a group with ks[g] == 0)
+ *   ks  [G] int32 on the device, each a multiple of 128, sum == K.  Only the
+ *       device reads it (graph-compatible).  A size that is negative, not a
+ *       multiple of 128, or a total other than K is recorded as
+ *       DG_ERR_INVALID_VALUE in the device status word; the kernel then uses
+ *       the K-blocks that exist (rounded down, clipped at K).
+ * 1 <= G <= 1024; M == 0 is a no-op.
+ */
+DG_API dg_status_t dg_k_grouped_fp8_gemm_nt_contiguous(const uint8_t *a, const float *sfa,
+                                                       int ld_sfa, const uint8_t *b,
+                                                       const float *sfb, void *d,
+                                                       const int32_t *ks, int G, int M, int N,
+                                                       int K, void *stream);
+
+/*
  * Per-token 1x128 activation quantiser (page 2 "技术特性": fine-grained
  * dynamic scaling; page 3 "核心功能": block-wise scaling): produces the A
  * operand and sfa of the GEMMs above from BF16 activations.  For each row m

@@ -58,10 +58,12 @@ def lib() -> ctypes.CDLL:
     L.dg_fp8_gemm_nt.argtypes = [P, P, I, P, P, P, I, I, I, P]
     L.dg_m_grouped_fp8_gemm_nt_contiguous.argtypes = [P, P, I, P, P, P, P, I, I, I, I, P]
     L.dg_m_grouped_fp8_gemm_nt_masked.argtypes = [P, P, I, P, P, P, P, I, I, I, I, P]
+    L.dg_k_grouped_fp8_gemm_nt_contiguous.argtypes = [P, P, I, P, P, P, P, I, I, I, I, P]
     L.dg_per_token_cast_to_fp8.argtypes = [P, P, P, I, I, I, P]
     L.dg_per_token_cast_to_fp8_masked.argtypes = [P, P, P, I, P, I, I, I, P]
     for f in ("dg_fp8_gemm_nt", "dg_m_grouped_fp8_gemm_nt_contiguous",
-              "dg_m_grouped_fp8_gemm_nt_masked", "dg_per_token_cast_to_fp8",
+              "dg_m_grouped_fp8_gemm_nt_masked", "dg_k_grouped_fp8_gemm_nt_contiguous",
+              "dg_per_token_cast_to_fp8",
               "dg_per_token_cast_to_fp8_masked"):
         getattr(L, f).restype = I
     L.dg_get_m_alignment_for_contiguous_layout.argtypes = []
@@ -153,6 +155,25 @@ def dg_m_grouped_fp8_gemm_nt_masked(a, sfa, b, sfb, d, masked_m, stream=None):
     _check(st, "dg_m_grouped_fp8_gemm_nt_masked")
     return d
 
+
+
+def dg_k_grouped_fp8_gemm_nt_contiguous(a, sfa, b, sfb, d, ks, stream=None):
+    """K-grouped GEMM (groups contiguous along K).  a uint8 [M,K]; sfa float32
+    [KB, ld_sfa]; b uint8 [N,K]; sfb float32 [NB,KB]; d bfloat16 [G,M,N];
+    ks int32 [G] (device), multiples of 128 adding up to K."""
+    import torch
+    M, K = a.shape
+    N = b.shape[-2]
+    G = ks.shape[0]
+    if tuple(d.shape) != (G, M, N):
+        raise ValueError(f"d must be [G, M, N] = {(G, M, N)}")
+    st = lib().dg_k_grouped_fp8_gemm_nt_contiguous(
+        _req(a, torch.uint8, "a", 2), _req(sfa, torch.float32, "sfa", 2), sfa.shape[-1],
+        _req(b, torch.uint8, "b", (2, 3)), _req(sfb, torch.float32, "sfb", (2, 3)),
+        _req(d, torch.bfloat16, "d", 3), _req(ks, torch.int32, "ks", 1), G, M, N, K,
+        _stream_handle(stream))
+    _check(st, "dg_k_grouped_fp8_gemm_nt_contiguous")
+    return d
 
 # --------------------------------------------------------------------------- quantisers
 def dg_per_token_cast_to_fp8(x, q, sfa, stream=None):

@@ -442,6 +442,47 @@ dg_status_t dg_m_grouped_fp8_gemm_nt_masked(const uint8_t *a, const float *sfa, 
     return launch<256, false, 4, dg::kMasked>(ma, mb, p, grid, 1, 1, s);
 }
 
+dg_status_t dg_k_grouped_fp8_gemm_nt_contiguous(const uint8_t *a, const float *sfa, int ld_sfa,
+                                                const uint8_t *b, const float *sfb, void *d,
+                                                const int32_t *ks, int G, int M, int N, int K,
+                                                void *stream) {
+    dg_status_t st = check_common(a, sfa, ld_sfa, b, sfb, d, M, N, K);
+    if (st != DG_SUCCESS) return st;
+    if (!ks || G <= 0) return DG_ERR_INVALID_VALUE;
+    if (G > dg::kMaxGroups) return DG_ERR_UNSUPPORTED_SHAPE;
+    const DeviceInfo *info = nullptr;
+    if ((st = device_info(&info)) != DG_SUCCESS) return st;
+    if (M == 0) return DG_SUCCESS;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    dg::Params p = base_params(sfa, ld_sfa, sfb, d, M, N, K, G, info);
+    p.ks = ks;
+    CUtensorMap ma, mb;
+    if ((st = make_map(&ma, a, K, M, 1, 128)) != DG_SUCCESS) return st;
+    // The tile grid does not depend on the group sizes (they only set each
+    // tile's K range, read on the device): G x token blocks x weight blocks.
+    if (N <= 128 || M <= 128) {
+        const int bn = N <= 128 ? 128 : 256;
+        const long long tiles = static_cast<long long>(G) * ((M + 127) / 128) * ((N + bn - 1) / bn);
+        const int grid = tiles < info->num_sms ? static_cast<int>(tiles) : info->num_sms;
+        if ((st = make_map(&mb, b, K, N, 1, bn)) != DG_SUCCESS) return st;
+        if (bn == 128) return launch<128, false, 6, dg::kKGrouped>(ma, mb, p, grid, 1, 1, s);
+        return launch<256, false, 4, dg::kKGrouped>(ma, mb, p, grid, 1, 1, s);
+    }
+    // CTA pairs: 256 x bn tiles (tcgen05.mma.cta_group::2), as for large dense GEMMs
+    const long long row_pairs = static_cast<long long>(G) * ((M + 255) / 256);
+    const int pm224 = max_active_clusters<224, false, 6, dg::kKGrouped, 2>(2);
+    const int pm256 = max_active_clusters<256, false, 6, dg::kKGrouped, 2>(2);
+    const int bn = pair_efficiency(row_pairs, N, 224, pm224) > pair_efficiency(row_pairs, N, 256, pm256) + 1e-9
+                       ? 224 : 256;
+    const int pairs_max = bn == 224 ? pm224 : pm256;
+    if (pairs_max <= 0) return cuda_fail(cudaErrorInvalidConfiguration, "no resident CTA pair");
+    const long long tiles = row_pairs * ((N + bn - 1) / bn);
+    const int pairs = tiles < pairs_max ? static_cast<int>(tiles) : pairs_max;
+    if ((st = make_map(&mb, b, K, N, 1, bn / 2)) != DG_SUCCESS) return st;
+    if (bn == 224) return launch<224, false, 6, dg::kKGrouped, 2>(ma, mb, p, 2 * pairs, 1, 2, s);
+    return launch<256, false, 6, dg::kKGrouped, 2>(ma, mb, p, 2 * pairs, 1, 2, s);
+}
+
 int dg_get_m_alignment_for_contiguous_layout(void) { return 128; }
 
 size_t dg_get_tma_aligned_size(size_t n, size_t elem_bytes) {

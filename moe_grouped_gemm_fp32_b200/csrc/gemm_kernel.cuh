@@ -54,7 +54,7 @@
 
 namespace dg {
 
-enum Layout : int { kDense = 0, kContiguous = 1, kMasked = 2 };
+enum Layout : int { kDense = 0, kContiguous = 1, kMasked = 2, kKGrouped = 3 };
 
 constexpr int kBlockK = 128;         // K-block (one 128-byte swizzled row of FP8)
 constexpr int kTileX = 128;          // MMA M per CTA (TMEM lanes)
@@ -77,7 +77,7 @@ constexpr int kTokBox = 32;          // swap mode: token rows per TMA box
 enum StatusCode : unsigned { kStatusInvalid = 1u, kStatusTimeout = 6u };
 enum Site : unsigned {
     kSiteProducerEmpty = 1, kSiteMmaTmemEmpty = 2, kSiteMmaFull = 3, kSitePromoFull = 4,
-    kSiteTeardownLoads = 5, kSiteTeardownMma = 6, kSiteBadGroup = 7, kSiteBadMask = 8
+    kSiteTeardownLoads = 5, kSiteTeardownMma = 6, kSiteBadGroup = 7, kSiteBadMask = 8, kSiteBadKs = 10
 };
 
 struct Params {
@@ -86,6 +86,7 @@ struct Params {
     __nv_bfloat16 *d;
     const int32_t *m_indices;   // contiguous
     const int32_t *masked_m;    // masked
+    const int32_t *ks;          // K-grouped: K columns per group (device)
     unsigned *status;           // device status word
     long long timeout_cycles;
     int ld_sfa;
@@ -159,6 +160,9 @@ struct Tile {
     int n0;      // first weight row
     int ntok;    // token rows of this tile that exist: min(rows per tile, tok_end - tok0)
     int store;   // CTA-pair tiles: bit r set = CTA r of the pair stores its rows
+    int b_grp;   // B tensor-map outer coordinate and sfb group (K-grouped: 0)
+    int kb0;     // the tile's K-blocks [kb0, kb1) (K-grouped: its group's)
+    int kb1;
 };
 
 template <int kBN, bool kSwap, int kLayout, int kCtaGroup>
@@ -184,6 +188,7 @@ struct TileMap {
     __device__ static int count(const Params &p, const int *prefix) {
         const int nw = (p.N + kWRows - 1) / kWRows;
         if (kLayout == kMasked) return prefix[p.G];
+        if (kLayout == kKGrouped) return p.G * ((p.M + kTokRows - 1) / kTokRows) * nw;
         if (kPairedGroups) {
             const int npairs = (p.M / kTileX + 1) / 2;
             return (npairs + prefix[kMaxGroups]) * nw;
@@ -196,6 +201,33 @@ struct TileMap {
     __device__ static bool decode(int t, const Params &p, const int *prefix, Tile &tl) {
         const int nw = (p.N + kWRows - 1) / kWRows;
         int tb, wb;
+        tl.kb0 = 0;
+        tl.kb1 = p.num_kb;
+        if (kLayout == kKGrouped) {
+            // group-major; inside a group the dense raster (bands of token blocks)
+            const int nt = (p.M + kTokRows - 1) / kTokRows;
+            const int g = t / (nt * nw);
+            const int local_t = t - g * nt * nw;
+            const int per_band = kRasterM * nw;
+            const int band = local_t / per_band;
+            const int first = band * kRasterM;
+            const int width = min(kRasterM, nt - first);
+            const int local = local_t - band * per_band;
+            tb = first + local % width;
+            wb = local / width;
+            tl.g = g;
+            tl.b_grp = 0;
+            tl.a_grp = 0;
+            tl.tok0 = tb * kTokRows;
+            tl.a_row = tl.tok0;
+            tl.tok_end = p.M;
+            tl.n0 = wb * kWRows;
+            tl.ntok = min(kTokRows, p.M - tl.tok0);
+            tl.store = 3;
+            tl.kb0 = prefix[g];
+            tl.kb1 = prefix[g + 1];
+            return true;
+        }
         if (kLayout == kMasked) {
             int lo = 0, hi = p.G - 1;                // last g with prefix[g] <= t
             while (lo < hi) {
@@ -211,6 +243,7 @@ struct TileMap {
             wb = local / ntb;
             tb = local - wb * ntb;
             tl.g = g;
+            tl.b_grp = g;
             tl.a_grp = g;
             tl.tok0 = tb * kTokRows;
             tl.a_row = tl.tok0;
@@ -244,6 +277,7 @@ struct TileMap {
                 store = 2;
             }
             tl.g = g;
+            tl.b_grp = g;
             tl.tok0 = pair * kTokRows;
             tl.a_row = tl.tok0;
             tl.a_grp = 0;
@@ -273,12 +307,14 @@ struct TileMap {
         tl.n0 = wb * kWRows;
         tl.ntok = min(kTokRows, p.M - tl.tok0);
         tl.g = 0;
+        tl.b_grp = 0;
         tl.store = 3;
         if (kLayout == kContiguous) {
             const int g = __ldg(p.m_indices + tl.tok0);
             if (g < 0) return false;
             if (g >= p.G) return false;     // recorded by the producer
             tl.g = g;
+            tl.b_grp = g;
         }
         return true;
     }
@@ -339,7 +375,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
     constexpr bool kSplitK = kSwap && kLayout == kDense && kBN <= 128;
     // the producer starts loading before the set-up barrier when nothing it
     // needs comes from other warps (not for CTA pairs or the masked layout)
-    constexpr bool kEarly = kCtaGroup == 1 && kLayout != kMasked;
+    constexpr bool kEarly = kCtaGroup == 1 && kLayout != kMasked && kLayout != kKGrouped;
     using L = SmemLayout<kBN, kSwap, kStages, kCtaGroup, kSplitK>;
     using TM = TileMap<kBN, kSwap, kLayout, kCtaGroup>;
     static_assert(kBN == 64 || kBN == 128 || kBN == 160 || kBN == 224 || kBN == 256, "tile N");
@@ -434,6 +470,37 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
         }
         if (lane == 0) prefix[p.G] = carry;
     }
+    if (kLayout == kKGrouped && warp == kPromoWarp0) {
+        // exclusive prefix of K-blocks per group (group g owns [prefix[g], prefix[g+1])).
+        // A size that is negative or not a multiple of 128, or a running total past
+        // K, is recorded and clipped: such a group gets only the K-blocks that exist.
+        int carry = 0;
+        for (int base = 0; base < p.G; base += 32) {
+            const int g = base + lane;
+            int kbs = 0;
+            if (g < p.G) {
+                const int kg = __ldg(p.ks + g);
+                if (kg < 0 || kg % kBlockK != 0) record_status(p.status, kStatusInvalid, kSiteBadKs);
+                kbs = kg > 0 ? kg / kBlockK : 0;
+            }
+            int incl = kbs;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int v = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += v;
+            }
+            if (g < p.G) {
+                const int lo = carry + incl - kbs, hi = carry + incl;
+                if (hi > p.num_kb) record_status(p.status, kStatusInvalid, kSiteBadKs);
+                prefix[g] = min(lo, p.num_kb);
+            }
+            carry += __shfl_sync(0xffffffffu, incl, 31);
+        }
+        if (lane == 0) {
+            if (carry != p.num_kb) record_status(p.status, kStatusInvalid, kSiteBadKs);   // sizes must add up to K
+            prefix[p.G] = min(carry, p.num_kb);
+        }
+    }
     if (TM::kPairedGroups && warp == kPromoWarp0) {
         // pairs of 128-row blocks whose groups differ: they get a second pass
         const int nblk = p.M / kTileX, npairs = (nblk + 1) / 2;
@@ -519,7 +586,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
                     continue;
                 }
                 const float *sfa_g = p.sfa + (kLayout == kMasked ? static_cast<size_t>(tl.g) * p.num_kb * p.ld_sfa : 0);
-                const float *sfb_g = p.sfb + static_cast<size_t>(tl.g) * p.num_nb * p.num_kb;
+                const float *sfb_g = p.sfb + static_cast<size_t>(tl.b_grp) * p.num_nb * p.num_kb;
                 const int wblk0 = tl.n0 / 128;
                 // swap mode fetches only the tile's token rows, in boxes of kTokBox rows
                 const int nload = kSwap ? (tl.ntok + kTokBox - 1) / kTokBox : 1;
@@ -532,7 +599,8 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
                 // operand bytes on this CTA's full barrier (a pair's MMA CTA counts both CTAs')
                 const uint32_t op_bytes = kPair ? (mma_cta ? 2u * (L::kXBytes + y_bytes) : 0u)
                                                 : L::kXBytes + y_bytes;
-                for (int kb = kb_begin; kb < kb_end; ++kb) {
+                const int kb_lo = max(kb_begin, tl.kb0), kb_hi = min(kb_end, tl.kb1);
+                for (int kb = kb_lo; kb < kb_hi; ++kb) {
                     if (!wait(empty_bar(stage), phase ^ 1u, kSiteProducerEmpty)) { ok = false; break; }
                     if (kSwap && !wait(sempty_bar(sslot), sphase ^ 1u, kSiteProducerEmpty)) { ok = false; break; }
                     const uint32_t sx = s_base + stage * L::kStageBytes;
@@ -558,7 +626,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
                         ptx::bulk_load(slot, sfa_g + static_cast<size_t>(kb) * p.ld_sfa + sa_row0, sa_bytes,
                                        scale_bar);
                     if (kSwap) {
-                        ptx::tma_load_3d(sx, &tm_b, full_bar(stage), kb * kBlockK, tl.n0, tl.g);
+                        ptx::tma_load_3d(sx, &tm_b, full_bar(stage), kb * kBlockK, tl.n0, tl.b_grp);
                         for (int i = 0; i < nload; ++i)
                             ptx::tma_load_3d(sy + i * kTokBox * kBlockK, &tm_a, full_bar(stage), kb * kBlockK,
                                              tl.a_row + i * kTokBox, tl.a_grp);
@@ -567,10 +635,10 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
                         const uint32_t fb = leader_addr(full_bar(stage));
                         ptx::tma_load_3d_pair(sx, &tm_a, fb, kb * kBlockK, tl.a_row + my_row0, tl.a_grp);
                         ptx::tma_load_3d_pair(sy, &tm_b, fb, kb * kBlockK,
-                                              tl.n0 + static_cast<int>(pair_rank) * L::kYRows, tl.g);
+                                              tl.n0 + static_cast<int>(pair_rank) * L::kYRows, tl.b_grp);
                     } else {
                         ptx::tma_load_3d(sx, &tm_a, full_bar(stage), kb * kBlockK, tl.a_row, tl.a_grp);
-                        ptx::tma_load_3d(sy, &tm_b, full_bar(stage), kb * kBlockK, tl.n0, tl.g);
+                        ptx::tma_load_3d(sy, &tm_b, full_bar(stage), kb * kBlockK, tl.n0, tl.b_grp);
                     }
                     ++issued;
                     if (++stage == kStages) { stage = 0; phase ^= 1u; }
@@ -612,7 +680,8 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
                 if (!TM::decode(t, p, prefix, tl)) continue;
                 const uint32_t idesc = f8_idesc(kTileX * kCtaGroup,
                                                 kSwap ? (tl.ntok + kTokBox - 1) / kTokBox * kTokBox : kBN);
-                for (int kb = kb_begin; kb < kb_end; ++kb) {
+                const int kb_lo = max(kb_begin, tl.kb0), kb_hi = min(kb_end, tl.kb1);
+                for (int kb = kb_lo; kb < kb_hi; ++kb) {
                     if (!wait(tempty_bar(buf), tphase ^ 1u, kSiteMmaTmemEmpty)) { ok = false; break; }
                     if (!wait(full_bar(stage), phase, kSiteMmaFull)) { ok = false; break; }
                     ptx::tc_fence_after();
@@ -685,7 +754,8 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
             Tile tl;
             if (!TM::decode(t, p, prefix, tl)) continue;
             const int ncols = (tl.ntok + kTokBox - 1) / kTokBox * kTokBox;
-            for (int kb = kb_begin; kb < kb_end; ++kb) {
+            const int kb_lo = max(kb_begin, tl.kb0), kb_hi = min(kb_end, tl.kb1);
+            for (int kb = kb_lo; kb < kb_hi; ++kb) {
                 if (!wait(sfull_bar(sslot), sphase, kSitePromoFull)) { ok = false; break; }
                 float *sl = slots + sslot * L::kSlotFloats;
                 const float sb = sl[L::kScaleRows];
@@ -749,7 +819,8 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
             const int ncols = kSwap ? (tl.ntok + kTokBox - 1) / kTokBox * kTokBox : kBN;
             const int nvalid = kSwap ? (ncols / kChunk - half + 1) / 2 : kChunks;
             const int wblk0 = tl.n0 / 128;
-            for (int kb = kb_begin; kb < kb_end; ++kb) {
+            const int kb_lo = max(kb_begin, tl.kb0), kb_hi = min(kb_end, tl.kb1);
+            for (int kb = kb_lo; kb < kb_hi; ++kb) {
                 // the K-block's scales: normal mode, visible once the stage's full
                 // barrier completed; swap mode, once the scale-prep warp is done
                 if (!wait(kSwap ? sready_bar(sslot) : full_bar(stage), kSwap ? sphase : phase,
@@ -886,7 +957,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
             have_tile = true;
             if (clustered) break;   // one tile; reduced below
             // ------------------------------------------------ epilogue (direct)
-            const size_t row_base = kLayout == kMasked ? static_cast<size_t>(tl.g) * p.M : 0;
+            const size_t row_base = (kLayout == kMasked || kLayout == kKGrouped) ? static_cast<size_t>(tl.g) * p.M : 0;
             if (!kSwap) {
                 if (tok_ok) {
                     __nv_bfloat16 *drow = p.d + (row_base + my_tok) * static_cast<size_t>(p.N);
@@ -962,7 +1033,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
         if (have_tile) {
             const float4 *recv = reinterpret_cast<const float4 *>(smem + L::kRecvOffset);
             const Tile &tl = last_tile;
-            const size_t row_base = kLayout == kMasked ? static_cast<size_t>(tl.g) * p.M : 0;
+            const size_t row_base = (kLayout == kMasked || kLayout == kKGrouped) ? static_cast<size_t>(tl.g) * p.M : 0;
             const int tid = (warp - kPromoWarp0) * 32 + lane;        // 0..255
             const int my_rows = min(rows_per, kTileX - static_cast<int>(my_rank) * rows_per);
             const int groups = (tl.ntok + 3) / 4;

@@ -22,6 +22,7 @@ class DeviceProblem:
         self.sfb = t(prob.sfb)
         self.m_indices = t(prob.m_indices) if prob.m_indices is not None else None
         self.masked_m = t(prob.masked_m) if prob.masked_m is not None else None
+        self.ks = t(prob.ks) if getattr(prob, "ks", None) is not None else None
         self.d = torch.empty(prob.d_shape(), dtype=torch.bfloat16, device=device)
 
     def fill_sentinel(self):
@@ -34,6 +35,9 @@ class DeviceProblem:
         elif p.layout == "contiguous":
             dg.dg_m_grouped_fp8_gemm_nt_contiguous(self.a, self.sfa, self.b, self.sfb, self.d,
                                                    self.m_indices, stream)
+        elif p.layout == "k_grouped":
+            dg.dg_k_grouped_fp8_gemm_nt_contiguous(self.a, self.sfa, self.b[0], self.sfb[0], self.d,
+                                                   self.ks, stream)
         else:
             dg.dg_m_grouped_fp8_gemm_nt_masked(self.a, self.sfa, self.b, self.sfb, self.d,
                                                self.masked_m, stream)
@@ -42,7 +46,7 @@ class DeviceProblem:
 
 def valid_mask(prob) -> np.ndarray:
     """Boolean mask over D of the rows the method computes."""
-    if prob.layout == "dense":
+    if prob.layout in ("dense", "k_grouped"):
         return np.ones(prob.d_shape(), bool)
     if prob.layout == "contiguous":
         return np.broadcast_to((prob.m_indices >= 0)[:, None], prob.d_shape())
