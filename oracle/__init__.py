@@ -10,6 +10,7 @@ definition for tiny shapes.
 
 Definition (DeepGEMM pages, page 2 "技术特性" and page 3 "核心功能"):
     D[m,n] = sum_kb sA[m,kb] * sB[n//128,kb] * sum_{k in kb} A[m,k] * B[n,k]
+BF16 GEMM (page 3 "核心功能"): D = sum_k A[m,k] * B[n,k], no block scales.
 K-grouped (page 3 "核心功能", k_grouped_gemm): group g sums only over its own
 ks[g] consecutive K columns, D[g] = the same sum over those K-blocks.
 Quantiser (page 2 "技术特性", dynamic fine-grained scaling): per row and
@@ -66,6 +67,8 @@ def _load():
         lib.oracle_k_grouped.restype = ctypes.c_int
         lib.oracle_k_grouped_points.argtypes = [P, P, L, P, P, P, L, L, L, L, L, P, P, P, P]
         lib.oracle_k_grouped_points.restype = ctypes.c_int
+        lib.oracle_bf16_gemm_nt.argtypes = [ctypes.c_int, P, P, P, P, L, L, L, L, P]
+        lib.oracle_bf16_gemm_nt.restype = ctypes.c_int
         lib.oracle_e4m3_encode.argtypes = [ctypes.c_float]
         lib.oracle_e4m3_encode.restype = ctypes.c_uint8
         lib.oracle_quantize_1x128.argtypes = [P, L, L, P, P, L]
@@ -139,6 +142,23 @@ def gemm_k_grouped(a, sfa, ld_sfa, b, sfb, ks, M, N, K) -> np.ndarray:
     rc = _load().oracle_k_grouped(_p(a), _p(sfa), ld_sfa, _p(b), _p(sfb), _p(ks), G, M, N, K, _p(d))
     if rc:
         raise ValueError(f"oracle_k_grouped rejected the input (rc={rc})")
+    return d
+
+
+def gemm_bf16(layout: str, a_bits, b_bits, M, N, K, G=1, m_indices=None, masked_m=None,
+              fill: float = np.nan) -> np.ndarray:
+    """BF16 NT GEMM on raw BF16 bit patterns (uint16): dense [M,N],
+    contiguous [M_total,N] (padding rows = fill), masked [G,Mmax,N] (rows past
+    masked_m = fill).  FP64 accumulation of exact products."""
+    a, b = _c(a_bits, np.uint16), _c(b_bits, np.uint16)
+    mi = None if m_indices is None else _c(m_indices, np.int32)
+    mm = None if masked_m is None else _c(masked_m, np.int32)
+    shape = (G, M, N) if layout == "masked" else (M, N)
+    d = np.full(shape, fill, dtype=np.float64)
+    rc = _load().oracle_bf16_gemm_nt(_LAYOUT_CODE[layout], _p(a), _p(b), _p(mi), _p(mm),
+                                     G, M, N, K, _p(d))
+    if rc:
+        raise ValueError(f"oracle_bf16_gemm_nt rejected the input (rc={rc})")
     return d
 
 

@@ -40,7 +40,8 @@
  * against exact integer arithmetic; identity and zero operands; scale
  * linearity; grouped == per-group dense; K-grouped: the groups' outputs sum
  * to the dense GEMM over all of K (exactly, for integer cases), one group ==
- * dense, an empty group gives zeros, brute force on tiny shapes.
+ * dense, an empty group gives zeros, brute force on tiny shapes.  BF16 GEMM:
+ * exact brute force, exact integer cases, grouped == per-group dense.
  */
 #include <math.h>
 #include <stdint.h>
@@ -281,6 +282,66 @@ int oracle_k_grouped_points(const uint8_t *a, const float *sfa, long ld_sfa,
                                             b + n * K + kb0 * ORC_BLOCK,
                                             sfb + (n / ORC_BLOCK) * KB + kb0, Kg, lut);
     }
+    return 0;
+}
+
+/* ------------------------------------------------------------------------
+ * BF16 GEMM (DeepGEMM page 3 "核心功能": FP8, FP4 and BF16 GEMMs), NT like
+ * the FP8 one, no block scales:
+ *
+ *   D[m,n] = sum_k A[m,k] * B[n,k]          (A [M,K], B [N,K] BF16, K-major)
+ *
+ * evaluated in FP64 (the BF16 values widened exactly; each product of two
+ * BF16 values is exact in FP64, the sum is FP64); callers round to BF16 or
+ * compare with a tolerance.  Layouts as for FP8: dense; M-grouped contiguous
+ * (row m uses B[m_indices[m]], rows with a negative index untouched); masked
+ * (a [G][Mmax][K], rows m < masked_m[g]).
+ * ------------------------------------------------------------------------ */
+static double bf16_value(uint16_t bits)
+{
+    union { uint32_t u; float f; } v;
+    v.u = (uint32_t)bits << 16;
+    return (double)v.f;
+}
+
+static double bf16_dot(const uint16_t *arow, const uint16_t *brow, long K)
+{
+    double acc = 0.0;
+    for (long k = 0; k < K; ++k)
+        acc += bf16_value(arow[k]) * bf16_value(brow[k]);
+    return acc;
+}
+
+/* layout 0 dense, 1 contiguous (m_indices), 2 masked (masked_m); rows_a is M,
+ * M_total or Mmax.  Output d [rows][N] (masked: [G][Mmax][N]); rows that the
+ * layout does not compute are left as they are. */
+int oracle_bf16_gemm_nt(int layout, const uint16_t *a, const uint16_t *b,
+                        const int32_t *m_indices, const int32_t *masked_m,
+                        long G, long rows_a, long N, long K, double *d)
+{
+    if (rows_a < 0 || N <= 0 || K <= 0 || G <= 0) return 1;
+    if (layout == 1)
+        for (long m = 0; m < rows_a; ++m)
+            if (m_indices[m] >= G) return 2;
+    if (layout == 2)
+        for (long g = 0; g < G; ++g)
+            if (masked_m[g] < 0 || masked_m[g] > rows_a) return 2;
+    long groups = layout == 2 ? G : 1;
+    #pragma omp parallel for collapse(2) schedule(dynamic, 1)
+    for (long g = 0; g < groups; ++g)
+        for (long m = 0; m < rows_a; ++m) {
+            long bg = 0;
+            if (layout == 1) {
+                if (m_indices[m] < 0) continue;
+                bg = m_indices[m];
+            } else if (layout == 2) {
+                if (m >= masked_m[g]) continue;
+                bg = g;
+            }
+            const uint16_t *arow = a + (g * rows_a + m) * K;
+            for (long n = 0; n < N; ++n)
+                d[(g * rows_a + m) * N + n] = bf16_dot(arow, b + (bg * N + n) * K, K);
+        }
     return 0;
 }
 

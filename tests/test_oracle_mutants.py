@@ -31,6 +31,10 @@ MUTANTS = {
         ("        off += Kg;\n", "        off += 0;\n"),
     "k-grouped: group's activation scales taken from K-block 0":
         ("sfa + kb0 * ld_sfa + m", "sfa + m"),
+    "bf16: mantissa shifted by one bit":
+        ("v.u = (uint32_t)bits << 16;", "v.u = (uint32_t)bits << 15;"),
+    "bf16: contiguous rows use group 0's weights":
+        ("                bg = m_indices[m];\n", "                bg = 0;\n"),
     "quantiser: scale amax / 240 (the E4M3 'fnuz' maximum)":
         ("float s = amax / 448.0f;", "float s = amax / 240.0f;"),
     "quantiser: encoder rounds ties away from zero":
@@ -52,6 +56,7 @@ def test_pins_catch_mutant(name, tmp_path):
     env = dict(os.environ, ORACLE_SO=str(so))
     r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
                         os.path.join(ROOT, "tests", "test_oracle.py"),
-                        os.path.join(ROOT, "tests", "test_oracle_quant.py")],
+                        os.path.join(ROOT, "tests", "test_oracle_quant.py"),
+                        os.path.join(ROOT, "tests", "test_oracle_bf16.py")],
                        cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
     assert r.returncode != 0, f"pins did not catch: {name}\n{r.stdout[-2000:]}"

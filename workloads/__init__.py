@@ -412,3 +412,117 @@ def make_quant_workload(name: str, seed_offset: int = 0) -> QuantProblem:
     if kind == "dense":
         return make_activations(w["M"], w["K"], seed, name=name)
     return make_activations_masked_uniform(w["G"], w["Mmax"], w["K"], seed, name=name)
+
+
+# ----------------------------------------------------------------------------- BF16 GEMM inputs
+BF16_NAN_BITS = 0x7FC0    # a BF16 NaN pattern, used to poison rows that must not be read
+
+
+@dataclasses.dataclass
+class BF16Problem:
+    """One BF16 NT GEMM problem (no block scales): raw BF16 bit patterns.
+    a: uint16 [rows, K] (masked: [G, Mmax, K]); b: uint16 [G, N, K]."""
+    layout: str                    # "dense" | "contiguous" | "masked"
+    M: int                         # dense: rows; contiguous: M_total; masked: Mmax
+    N: int
+    K: int
+    G: int
+    a: np.ndarray
+    b: np.ndarray
+    m_indices: Optional[np.ndarray] = None
+    masked_m: Optional[np.ndarray] = None
+    name: str = ""
+
+    def valid_rows(self) -> int:
+        if self.layout == "dense":
+            return self.M
+        if self.layout == "contiguous":
+            return int((self.m_indices >= 0).sum())
+        return int(self.masked_m.sum())
+
+    def groups_touched(self) -> int:
+        if self.layout == "dense":
+            return 1
+        if self.layout == "contiguous":
+            return int(len(np.unique(self.m_indices[self.m_indices >= 0])))
+        return int((self.masked_m > 0).sum())
+
+    def flops(self) -> float:
+        return 2.0 * self.valid_rows() * self.N * self.K
+
+    def bytes(self) -> float:
+        """Algorithmic bytes: A and D over valid rows, B of the touched groups."""
+        rows, g = self.valid_rows(), self.groups_touched()
+        return float(2 * rows * self.K + 2 * g * self.N * self.K + 2 * rows * self.N)
+
+    def d_shape(self):
+        if self.layout == "masked":
+            return (self.G, self.M, self.N)
+        return (self.M, self.N)
+
+
+def _bf16_bits(x32: np.ndarray) -> np.ndarray:
+    return torch.from_numpy(np.ascontiguousarray(x32)).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+
+
+def make_bf16_dense(M: int, N: int, K: int, seed: int, name: str = "") -> BF16Problem:
+    """A ~ N(0,1) [M,K], B ~ N(0,1) [N,K], rounded to BF16."""
+    rng = np.random.default_rng(seed)
+    a = _bf16_bits(_normal(rng, (M, K)))
+    b = _bf16_bits(_normal(rng, (N, K)))
+    return BF16Problem("dense", M, N, K, 1, a, b[None], name=name)
+
+
+def make_bf16_contiguous(counts, N: int, K: int, seed: int, name: str = "") -> BF16Problem:
+    """Contiguous layout: groups packed back to back, each padded to 128 rows;
+    padding rows hold BF16 NaN and m_indices -1."""
+    rng = np.random.default_rng(seed)
+    counts = [int(c) for c in counts]
+    G = len(counts)
+    padded = [(c + ALIGN_M - 1) // ALIGN_M * ALIGN_M for c in counts]
+    M_total = int(sum(padded))
+    a_all = _bf16_bits(_normal(rng, (sum(counts), K)))
+    b = _bf16_bits(_normal(rng, (G * N, K))).reshape(G, N, K)
+    a = np.full((M_total, K), BF16_NAN_BITS, dtype=np.uint16)
+    m_idx = np.full((M_total,), -1, dtype=np.int32)
+    src = dst = 0
+    for g, (c, p) in enumerate(zip(counts, padded)):
+        a[dst:dst + c] = a_all[src:src + c]
+        m_idx[dst:dst + c] = g
+        src += c
+        dst += p
+    return BF16Problem("contiguous", M_total, N, K, G, a, b, m_indices=m_idx, name=name)
+
+
+def make_bf16_masked(masked_m, Mmax: int, N: int, K: int, seed: int, name: str = "") -> BF16Problem:
+    """Masked layout: a [G, Mmax, K]; rows >= masked_m[g] hold BF16 NaN."""
+    rng = np.random.default_rng(seed)
+    masked_m = np.asarray(masked_m, dtype=np.int32)
+    G = len(masked_m)
+    a = _bf16_bits(_normal(rng, (G * Mmax, K))).reshape(G, Mmax, K)
+    b = _bf16_bits(_normal(rng, (G * N, K))).reshape(G, N, K)
+    for g in range(G):
+        a[g, masked_m[g]:] = BF16_NAN_BITS
+    return BF16Problem("masked", Mmax, N, K, G, a, b, masked_m=masked_m, name=name)
+
+
+BF16_WORKLOADS = {
+    "bf16_dense_large": dict(kind="dense", M=4096, N=7168, K=16384, seed=11),
+    "bf16_dense_decode_m64": dict(kind="dense", M=64, N=2112, K=7168, seed=12),
+    "bf16_contiguous_g4": dict(kind="contiguous", G=4, tokens=32768, N=4096, K=7168, seed=13),
+    "bf16_masked_g16": dict(kind="masked", G=16, Mmax=256, N=4096, K=7168, seed=14),
+}
+
+
+def make_bf16_workload(name: str, seed_offset: int = 0) -> BF16Problem:
+    w = dict(BF16_WORKLOADS[name])
+    kind = w.pop("kind")
+    seed = w.pop("seed") + seed_offset
+    if kind == "dense":
+        return make_bf16_dense(w["M"], w["N"], w["K"], seed, name=name)
+    rng = np.random.default_rng(seed)
+    if kind == "contiguous":
+        counts = rng.multinomial(w["tokens"], [1.0 / w["G"]] * w["G"])
+        return make_bf16_contiguous(counts, w["N"], w["K"], seed + 1000, name=name)
+    masked_m = rng.integers(0, w["Mmax"] + 1, size=w["G"]).astype(np.int32)
+    return make_bf16_masked(masked_m, w["Mmax"], w["N"], w["K"], seed + 1000, name=name)
