@@ -39,6 +39,8 @@ PAGES_NUMBER = {"dense_decode_m64": (1688.0, "GB/s")}
 UNIT = {"dense_tiny": "TFLOP/s", "dense_decode_m64": "GB/s", "dense_decode_m128": "GB/s",
         "dense_large": "TFLOP/s", "contiguous_g4": "TFLOP/s", "masked_g16": "GB/s",
         "kgrouped_g4": "TFLOP/s",
+        "bf16_dense_large": "TFLOP/s", "bf16_contiguous_g4": "TFLOP/s", "bf16_masked_g16": "GB/s",
+        "bf16_dense_decode_m64": "GB/s",
         "quant_tiny": "GB/s", "quant_tokens_32768": "GB/s", "quant_masked_g16": "GB/s"}
 # the kernel each workload times, and the sources whose hash keys its ncu summary
 KERNEL_SOURCES = {
@@ -47,6 +49,10 @@ KERNEL_SOURCES = {
                         "moe_grouped_gemm_fp32_b200/csrc/dg_api.cu"],
     "quant_1x128_kernel": ["moe_grouped_gemm_fp32_b200/csrc/quant_kernel.cuh",
                            "moe_grouped_gemm_fp32_b200/csrc/quant_api.cu"],
+    "bf16_gemm_kernel": ["moe_grouped_gemm_fp32_b200/csrc/bf16_kernel.cuh",
+                         "moe_grouped_gemm_fp32_b200/csrc/bf16_api.cu",
+                         "moe_grouped_gemm_fp32_b200/csrc/gemm_kernel.cuh",
+                         "moe_grouped_gemm_fp32_b200/csrc/ptx.cuh"],
 }
 FLUSH_BYTES = 512 << 20
 
@@ -55,8 +61,14 @@ def is_quant(workload: str) -> bool:
     return workload.startswith("quant_")
 
 
+def is_bf16(workload: str) -> bool:
+    return workload.startswith("bf16_")
+
+
 def kernel_name(workload: str) -> str:
-    return "quant_1x128_kernel" if is_quant(workload) else "fp8_gemm_kernel"
+    if is_quant(workload):
+        return "quant_1x128_kernel"
+    return "bf16_gemm_kernel" if is_bf16(workload) else "fp8_gemm_kernel"
 
 
 def kernel_source_hash(kernel: str = "fp8_gemm_kernel") -> str:
@@ -158,6 +170,8 @@ def rank_problem(workload: str, rank: int):
     import workloads as W
     if is_quant(workload):
         return W.make_quant_workload(workload, seed_offset=7919 * rank)
+    if is_bf16(workload):
+        return W.make_bf16_workload(workload, seed_offset=7919 * rank)
     if rank == 0:
         return W.make_workload(workload)
     spec = dict(W.WORKLOADS[workload])
@@ -224,6 +238,38 @@ class GemmCall:
         return self.d.numel() * self.d.element_size()
 
 
+class Bf16Call:
+    """Pinned BF16 operands, device output and the library call of one BF16 GEMM."""
+
+    def __init__(self, prob, dev):
+        import numpy as np
+        import torch
+        self.prob = prob
+        bf = lambda x: torch.from_numpy(np.ascontiguousarray(x).view(np.int16)).view(torch.bfloat16)
+        self.host = {"a": bf(prob.a).pin_memory(), "b": bf(prob.b).pin_memory()}
+        if prob.m_indices is not None:
+            self.host["m_indices"] = torch.from_numpy(prob.m_indices).pin_memory()
+        if prob.masked_m is not None:
+            self.host["masked_m"] = torch.from_numpy(prob.masked_m).pin_memory()
+        self.d = torch.empty(prob.d_shape(), dtype=torch.bfloat16, device=dev)
+        self.d_host = torch.empty(prob.d_shape(), dtype=torch.bfloat16).pin_memory()
+
+    def call(self, t, stream):
+        import moe_grouped_gemm_fp32_b200 as dg
+        if self.prob.layout == "dense":
+            dg.dg_bf16_gemm_nt(t["a"], t["b"][0], self.d, stream)
+        elif self.prob.layout == "contiguous":
+            dg.dg_m_grouped_bf16_gemm_nt_contiguous(t["a"], t["b"], self.d, t["m_indices"], stream)
+        else:
+            dg.dg_m_grouped_bf16_gemm_nt_masked(t["a"], t["b"], self.d, t["masked_m"], stream)
+
+    def read_back(self):
+        self.d_host.copy_(self.d, non_blocking=True)
+
+    def d2h_bytes(self) -> int:
+        return self.d.numel() * self.d.element_size()
+
+
 class QuantCall:
     """Pinned BF16 activations, device codes and scales, and the quantiser call."""
 
@@ -265,7 +311,7 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.set_device(dev)
     prob = rank_problem(args.workload, rank)
 
-    op = (QuantCall if is_quant(args.workload) else GemmCall)(prob, dev)
+    op = (QuantCall if is_quant(args.workload) else Bf16Call if is_bf16(args.workload) else GemmCall)(prob, dev)
     host = op.host
     devt = {k: v.to(dev, non_blocking=False) for k, v in host.items()}
     flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
@@ -368,6 +414,42 @@ def quant_cpu_baseline(prob, budget_s=10.0):
             "seconds_per_step": secs}
 
 
+def bf16_cpu_baseline(prob, unit, budget_s=10.0):
+    """The oracle BF16 GEMM as it stands (FP64 accumulation, all host cores) on
+    evenly spaced valid output rows, as many as fit ~budget_s, scaled linearly."""
+    import numpy as np
+    import oracle
+    oracle.build()
+    cores = len(os.sched_getaffinity(0))
+    if prob.layout == "masked":
+        sel = [(g, m) for g in range(prob.G) for m in range(int(prob.masked_m[g]))]
+    elif prob.layout == "contiguous":
+        sel = [(int(prob.m_indices[m]), m) for m in np.flatnonzero(prob.m_indices >= 0)]
+    else:
+        sel = [(0, m) for m in range(prob.M)]
+
+    def run(pick):
+        # one dense call per group over its picked rows (OpenMP over the rows)
+        for g in sorted({q[0] for q in pick}):
+            rows = [m for gg, m in pick if gg == g]
+            a = prob.a[g, rows] if prob.layout == "masked" else prob.a[rows]
+            oracle.gemm_bf16("dense", a, prob.b[g], len(rows), prob.N, prob.K)
+    probe = sel[:: max(1, len(sel) // 32)][:32]
+    t0 = time.perf_counter()
+    run(probe)
+    per_row = (time.perf_counter() - t0) / len(probe)
+    n = max(len(probe), min(len(sel), int(budget_s / max(per_row, 1e-9))))
+    pick = sel[:: max(1, len(sel) // n)][:n]
+    t0 = time.perf_counter()
+    run(pick)
+    dt = time.perf_counter() - t0
+    secs = dt * len(sel) / len(pick)
+    value = (prob.bytes() / secs / 1e9) if unit == "GB/s" else (prob.flops() / secs / 1e12)
+    return {"value": value, "unit": unit, "cores": cores, "kind": "oracle",
+            "sample": f"{len(pick)} of {len(sel)} valid output rows (all N columns), {dt:.1f} s, "
+                      f"scaled linearly to the whole workload", "seconds_per_step": secs}
+
+
 def cpu_baseline(prob, unit, budget_s=10.0):
     """The oracle as it stands (FP64, OpenMP over all host cores) on a bounded
     sample: whole problems repeated until ~budget_s, or a leading slice of the
@@ -376,6 +458,8 @@ def cpu_baseline(prob, unit, budget_s=10.0):
     import oracle
     if not hasattr(prob, "flops"):
         return quant_cpu_baseline(prob, budget_s)
+    if not hasattr(prob, "sfa"):
+        return bf16_cpu_baseline(prob, unit, budget_s)
     oracle.build()
     cores = len(os.sched_getaffinity(0))
     t0 = time.perf_counter()
@@ -473,6 +557,15 @@ def run_reference(args, rank, world):
 
 
 def shape_config(prob):
+    if hasattr(prob, "flops") and not hasattr(prob, "sfa"):   # BF16 GEMM
+        c = {"layout": prob.layout, "N": prob.N, "K": prob.K, "operands": "bf16"}
+        if prob.layout == "dense":
+            c["M"] = prob.M
+        elif prob.layout == "contiguous":
+            c.update(G=prob.G, M_total=prob.M, valid_rows=prob.valid_rows())
+        else:
+            c.update(G=prob.G, Mmax=prob.M, valid_rows=prob.valid_rows())
+        return c
     if not hasattr(prob, "flops"):          # quantiser inputs
         c = {"layout": prob.layout, "K": prob.K, "in": "bf16", "out": "e4m3 + f32 1x128 scales"}
         if prob.layout == "dense":
@@ -532,7 +625,8 @@ def main():
         achieved = prob.bytes() / (ms * 1e-3) / 1e9
     else:
         bound, runit = "tensor", "TFLOP/s"
-        peak = 2.0 * peaks["bf16_tflops"]          # FP8 dense = 2 x BF16 dense (nominal ratio)
+        # BF16: the measured BF16 peak; FP8 dense = 2 x BF16 dense (nominal ratio)
+        peak = peaks["bf16_tflops"] * (1.0 if is_bf16(args.workload) else 2.0)
         achieved = prob.flops() / (ms * 1e-3) / 1e12
     pages = PAGES_NUMBER.get(args.workload)
     line = {
@@ -540,6 +634,7 @@ def main():
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": (value / pages[0]) if pages and pages[1] == unit else None,
         "dtype": ("f32 (bf16 in, e4m3 out)" if is_quant(args.workload)
+                  else "bf16 (f32 accumulate, bf16 out)" if is_bf16(args.workload)
                   else "e4m3 (f32 accumulate, bf16 out)"),
         "data": "synthetic",
         "config": {"workload": args.workload, **shape_config(prob),
@@ -548,7 +643,7 @@ def main():
                    "gbps": prob.bytes() / (ms * 1e-3) / 1e9},
         "roofline": {"bound": bound, "achieved": achieved, "peak": peak, "unit": runit,
                      "frac": achieved / peak, "traffic": profiled_traffic(args.workload),
-                     "peak_source": f"{peak_src} ({'hbm_gbs' if bound == 'hbm' else '2 x bf16_tflops'})"},
+                     "peak_source": f"{peak_src} ({'hbm_gbs' if bound == 'hbm' else 'bf16_tflops' if is_bf16(args.workload) else '2 x bf16_tflops'})"},
         "e2e": {"value": metric_value(prob, unit, e2e_ms, world), "unit": unit,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": args.steps,

@@ -136,6 +136,34 @@ DG_API dg_status_t dg_k_grouped_fp8_gemm_nt_contiguous(const uint8_t *a, const f
                                                        int K, void *stream);
 
 /*
+ * BF16 GEMMs (page 3 "核心功能": FP8, FP4 and BF16 GEMM operations, in the same
+ * dense and m-grouped layouts):
+ *   D[m,n] = sum_k A[m,k] * B[n,k]    accumulated in FP32, stored as BF16 (RNE)
+ * A and B are BF16 (raw 16-bit patterns), K-major; no block scales.  Shape
+ * rules: K > 0, K % 8 == 0; N > 0, N % 8 == 0 (16-byte rows); M >= 0.
+ * Pointers, stream and error conventions as for the FP8 GEMMs.
+ *
+ * Dense: a [M, K], b [N, K], d [M, N].
+ */
+DG_API dg_status_t dg_bf16_gemm_nt(const void *a, const void *b, void *d, int M, int N, int K,
+                                   void *stream);
+
+/* Contiguous M-grouped BF16: a [M_total, K] (groups packed, each padded to 128
+ * rows), b [G, N, K], d [M_total, N], m_indices [M_total] int32 on the device
+ * with the same precondition and padding rules as the FP8 contiguous call.
+ * M_total % 128 == 0. */
+DG_API dg_status_t dg_m_grouped_bf16_gemm_nt_contiguous(const void *a, const void *b, void *d,
+                                                        const int32_t *m_indices, int M_total,
+                                                        int N, int K, int G, void *stream);
+
+/* Masked M-grouped BF16: a [G, Mmax, K], b [G, N, K], d [G, Mmax, N]; rows
+ * m < masked_m[g] computed, the others never written (graph-compatible, as for
+ * the FP8 masked call).  G <= 1024. */
+DG_API dg_status_t dg_m_grouped_bf16_gemm_nt_masked(const void *a, const void *b, void *d,
+                                                    const int32_t *masked_m, int G, int Mmax,
+                                                    int N, int K, void *stream);
+
+/*
  * Per-token 1x128 activation quantiser (page 2 "技术特性": fine-grained
  * dynamic scaling; page 3 "核心功能": block-wise scaling): produces the A
  * operand and sfa of the GEMMs above from BF16 activations.  For each row m

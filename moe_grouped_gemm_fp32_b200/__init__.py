@@ -59,10 +59,15 @@ def lib() -> ctypes.CDLL:
     L.dg_m_grouped_fp8_gemm_nt_contiguous.argtypes = [P, P, I, P, P, P, P, I, I, I, I, P]
     L.dg_m_grouped_fp8_gemm_nt_masked.argtypes = [P, P, I, P, P, P, P, I, I, I, I, P]
     L.dg_k_grouped_fp8_gemm_nt_contiguous.argtypes = [P, P, I, P, P, P, P, I, I, I, I, P]
+    L.dg_bf16_gemm_nt.argtypes = [P, P, P, I, I, I, P]
+    L.dg_m_grouped_bf16_gemm_nt_contiguous.argtypes = [P, P, P, P, I, I, I, I, P]
+    L.dg_m_grouped_bf16_gemm_nt_masked.argtypes = [P, P, P, P, I, I, I, I, P]
     L.dg_per_token_cast_to_fp8.argtypes = [P, P, P, I, I, I, P]
     L.dg_per_token_cast_to_fp8_masked.argtypes = [P, P, P, I, P, I, I, I, P]
     for f in ("dg_fp8_gemm_nt", "dg_m_grouped_fp8_gemm_nt_contiguous",
               "dg_m_grouped_fp8_gemm_nt_masked", "dg_k_grouped_fp8_gemm_nt_contiguous",
+              "dg_bf16_gemm_nt", "dg_m_grouped_bf16_gemm_nt_contiguous",
+              "dg_m_grouped_bf16_gemm_nt_masked",
               "dg_per_token_cast_to_fp8",
               "dg_per_token_cast_to_fp8_masked"):
         getattr(L, f).restype = I
@@ -173,6 +178,42 @@ def dg_k_grouped_fp8_gemm_nt_contiguous(a, sfa, b, sfb, d, ks, stream=None):
         _req(d, torch.bfloat16, "d", 3), _req(ks, torch.int32, "ks", 1), G, M, N, K,
         _stream_handle(stream))
     _check(st, "dg_k_grouped_fp8_gemm_nt_contiguous")
+    return d
+
+
+# --------------------------------------------------------------------------- BF16 GEMMs
+def dg_bf16_gemm_nt(a, b, d, stream=None):
+    """D[M,N] = A[M,K] * B[N,K]^T, all bfloat16 (FP32 accumulation)."""
+    import torch
+    M, K = a.shape
+    N = b.shape[-2]
+    st = lib().dg_bf16_gemm_nt(_req(a, torch.bfloat16, "a", 2), _req(b, torch.bfloat16, "b", (2, 3)),
+                               _req(d, torch.bfloat16, "d", 2), M, N, K, _stream_handle(stream))
+    _check(st, "dg_bf16_gemm_nt")
+    return d
+
+
+def dg_m_grouped_bf16_gemm_nt_contiguous(a, b, d, m_indices, stream=None):
+    """Contiguous M-grouped BF16 GEMM: a [M_total,K], b [G,N,K], d [M_total,N]."""
+    import torch
+    M_total, K = a.shape
+    G, N, _ = b.shape
+    st = lib().dg_m_grouped_bf16_gemm_nt_contiguous(
+        _req(a, torch.bfloat16, "a", 2), _req(b, torch.bfloat16, "b", 3), _req(d, torch.bfloat16, "d", 2),
+        _req(m_indices, torch.int32, "m_indices", 1), M_total, N, K, G, _stream_handle(stream))
+    _check(st, "dg_m_grouped_bf16_gemm_nt_contiguous")
+    return d
+
+
+def dg_m_grouped_bf16_gemm_nt_masked(a, b, d, masked_m, stream=None):
+    """Masked M-grouped BF16 GEMM: a [G,Mmax,K], b [G,N,K], d [G,Mmax,N]."""
+    import torch
+    G, Mmax, K = a.shape
+    N = b.shape[1]
+    st = lib().dg_m_grouped_bf16_gemm_nt_masked(
+        _req(a, torch.bfloat16, "a", 3), _req(b, torch.bfloat16, "b", 3), _req(d, torch.bfloat16, "d", 3),
+        _req(masked_m, torch.int32, "masked_m", 1), G, Mmax, N, K, _stream_handle(stream))
+    _check(st, "dg_m_grouped_bf16_gemm_nt_masked")
     return d
 
 # --------------------------------------------------------------------------- quantisers

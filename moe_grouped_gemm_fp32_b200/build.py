@@ -13,9 +13,9 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
-SOURCES = [os.path.join(CSRC, f) for f in ("dg_api.cu", "quant_api.cu")]
+SOURCES = [os.path.join(CSRC, f) for f in ("dg_api.cu", "quant_api.cu", "bf16_api.cu")]
 DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("gemm_kernel.cuh", "ptx.cuh", "quant_kernel.cuh",
-                                                  "api_common.h")] + [
+                                                  "bf16_kernel.cuh", "api_common.h")] + [
     os.path.join(ROOT, "include", "dg.h")]
 OUT = os.path.join(HERE, "_dg.so")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")

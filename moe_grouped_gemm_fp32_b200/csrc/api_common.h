@@ -4,6 +4,7 @@
 // nothing here is exported from the shared library.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -34,5 +35,14 @@ int debug_flags();
 
 // DG_VERBOSE=1 prints each launch's configuration to stderr.
 bool verbose();
+
+// Bounded-wait limit in clock cycles for kernels (DG_WAIT_TIMEOUT_CYCLES, read once).
+long long timeout_cycles();
+
+// 3-D tensor map {K, rows, groups} of elem_bytes-wide elements (1: uint8 E4M3,
+// 2: BF16), K innermost with a row stride of K elements; box {128 bytes of K,
+// box_rows, 1}; 128-byte swizzle; out-of-bounds elements read as zero.
+dg_status_t make_kmajor_map(CUtensorMap *m, const void *base, int elem_bytes, long long K,
+                            long long rows, long long groups, int box_rows);
 
 }  // namespace dg_host

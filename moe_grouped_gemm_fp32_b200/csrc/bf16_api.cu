@@ -1,0 +1,147 @@
+// bf16_api.cu -- host side of the BF16 GEMM entry points declared in
+// include/dg.h (dg_bf16_gemm_nt, dg_m_grouped_bf16_gemm_nt_contiguous,
+// dg_m_grouped_bf16_gemm_nt_masked): argument validation, TMA descriptors,
+// tile width by wave efficiency, launch.  Nothing here synchronises the host
+// or allocates memory.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdio>
+
+#include "dg.h"
+#include "api_common.h"
+#include "bf16_kernel.cuh"
+
+namespace {
+using namespace dg_host;
+
+dg_status_t check_bf16(const void *a, const void *b, const void *d, int rows, int N, int K) {
+    if (!a || !b || !d) return DG_ERR_INVALID_VALUE;
+    if (rows < 0 || N <= 0 || K <= 0) return DG_ERR_INVALID_VALUE;
+    // 16-byte row strides for TMA (K) and 16-byte output stores (N)
+    if (K % 8 != 0 || N % 8 != 0) return DG_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned16(a) || !aligned16(b) || !aligned16(d)) return DG_ERR_MISALIGNED;
+    if (static_cast<long long>(K) > (1LL << 30) || N > (1 << 30)) return DG_ERR_UNSUPPORTED_SHAPE;
+    return DG_SUCCESS;
+}
+
+dg::Params bf16_params(void *d, int rows, int N, int K, int G, const DeviceInfo *info) {
+    dg::Params p = {};
+    p.d = static_cast<__nv_bfloat16 *>(d);
+    p.status = info->status;
+    p.timeout_cycles = timeout_cycles();
+    p.M = rows;
+    p.N = N;
+    p.K = K;
+    p.G = G;
+    p.num_kb = (K + dg::kBf16BlockK - 1) / dg::kBf16BlockK;
+    p.num_nb = (N + 127) / 128;
+    p.split = 1;
+    p.debug_flags = debug_flags();
+    return p;
+}
+
+template <int kBN, int kStages, int kLayout>
+dg_status_t launch_bf16(const CUtensorMap &ma, const CUtensorMap &mb, const dg::Params &p, int grid,
+                        cudaStream_t stream) {
+    using L = dg::Bf16Smem<kBN, kStages>;
+    auto kernel = dg::bf16_gemm_kernel<kBN, kStages, kLayout>;
+    static bool configured[kMaxDevices] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (!configured[dev]) {
+        cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(bf16 smem)");
+        configured[dev] = true;
+    }
+    if (verbose())
+        std::fprintf(stderr, "[dg] bf16_gemm layout=%d bn=%d stages=%d grid=%d smem=%d\n", kLayout, kBN,
+                     kStages, grid, L::kAlloc);
+    kernel<<<grid, dg::kBf16Threads, L::kAlloc, stream>>>(ma, mb, p);
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? DG_SUCCESS : cuda_fail(e, "bf16_gemm_kernel launch");
+}
+
+// tile width: N <= 128 -> 128; otherwise 224 or 256, whichever wastes less of
+// the last wave and of the last weight-tile's columns
+int pick_bn(long long token_blocks, int N, int num_sms) {
+    if (N <= 128) return 128;
+    auto eff = [&](int bn) {
+        const long long nt = (N + bn - 1) / bn;
+        const long long tiles = token_blocks * nt;
+        const long long waves = (tiles + num_sms - 1) / num_sms;
+        return (static_cast<double>(N) / (nt * bn)) * (static_cast<double>(tiles) / (waves * num_sms));
+    };
+    return eff(224) > eff(256) + 1e-9 ? 224 : 256;
+}
+
+template <int kLayout>
+dg_status_t dispatch(const CUtensorMap &ma, const void *b, int N, int K, int G, const dg::Params &p,
+                     long long tiles_hint_blocks, int grid_cap, cudaStream_t s) {
+    const int bn = pick_bn(tiles_hint_blocks, N, grid_cap);
+    CUtensorMap mb;
+    dg_status_t st = make_kmajor_map(&mb, b, 2, K, N, G, bn);
+    if (st != DG_SUCCESS) return st;
+    const long long tiles = tiles_hint_blocks * ((N + bn - 1) / bn);
+    const int grid = tiles < grid_cap ? static_cast<int>(tiles > 0 ? tiles : 1) : grid_cap;
+    if (bn == 128) return launch_bf16<128, 6, kLayout>(ma, mb, p, grid, s);
+    if (bn == 224) return launch_bf16<224, 4, kLayout>(ma, mb, p, grid, s);
+    return launch_bf16<256, 4, kLayout>(ma, mb, p, grid, s);
+}
+
+}  // namespace
+
+extern "C" {
+
+dg_status_t dg_bf16_gemm_nt(const void *a, const void *b, void *d, int M, int N, int K, void *stream) {
+    dg_status_t st = check_bf16(a, b, d, M, N, K);
+    if (st != DG_SUCCESS) return st;
+    const DeviceInfo *info = nullptr;
+    if ((st = device_info(&info)) != DG_SUCCESS) return st;
+    if (M == 0) return DG_SUCCESS;
+    const dg::Params p = bf16_params(d, M, N, K, 1, info);
+    CUtensorMap ma;
+    if ((st = make_kmajor_map(&ma, a, 2, K, M, 1, 128)) != DG_SUCCESS) return st;
+    return dispatch<dg::kDense>(ma, b, N, K, 1, p, (M + 127) / 128, info->num_sms,
+                                static_cast<cudaStream_t>(stream));
+}
+
+dg_status_t dg_m_grouped_bf16_gemm_nt_contiguous(const void *a, const void *b, void *d,
+                                                 const int32_t *m_indices, int M_total, int N, int K,
+                                                 int G, void *stream) {
+    dg_status_t st = check_bf16(a, b, d, M_total, N, K);
+    if (st != DG_SUCCESS) return st;
+    if (!m_indices || G <= 0) return DG_ERR_INVALID_VALUE;
+    if (M_total % 128 != 0) return DG_ERR_UNSUPPORTED_SHAPE;
+    const DeviceInfo *info = nullptr;
+    if ((st = device_info(&info)) != DG_SUCCESS) return st;
+    if (M_total == 0) return DG_SUCCESS;
+    dg::Params p = bf16_params(d, M_total, N, K, G, info);
+    p.m_indices = m_indices;
+    CUtensorMap ma;
+    if ((st = make_kmajor_map(&ma, a, 2, K, M_total, 1, 128)) != DG_SUCCESS) return st;
+    return dispatch<dg::kContiguous>(ma, b, N, K, G, p, M_total / 128, info->num_sms,
+                                     static_cast<cudaStream_t>(stream));
+}
+
+dg_status_t dg_m_grouped_bf16_gemm_nt_masked(const void *a, const void *b, void *d,
+                                             const int32_t *masked_m, int G, int Mmax, int N, int K,
+                                             void *stream) {
+    dg_status_t st = check_bf16(a, b, d, Mmax, N, K);
+    if (st != DG_SUCCESS) return st;
+    if (!masked_m || G <= 0) return DG_ERR_INVALID_VALUE;
+    if (G > dg::kMaxGroups) return DG_ERR_UNSUPPORTED_SHAPE;
+    const DeviceInfo *info = nullptr;
+    if ((st = device_info(&info)) != DG_SUCCESS) return st;
+    if (Mmax == 0) return DG_SUCCESS;
+    dg::Params p = bf16_params(d, Mmax, N, K, G, info);
+    p.masked_m = masked_m;
+    CUtensorMap ma;
+    if ((st = make_kmajor_map(&ma, a, 2, K, Mmax, G, 128)) != DG_SUCCESS) return st;
+    // the tile count lives on the device: a persistent grid of one CTA per SM;
+    // the tile width assumes every group full (the workload's upper bound)
+    return dispatch<dg::kMasked>(ma, b, N, K, G, p, static_cast<long long>(G) * ((Mmax + 127) / 128),
+                                 info->num_sms, static_cast<cudaStream_t>(stream)) ;
+}
+
+}  // extern "C"

@@ -1,0 +1,282 @@
+// bf16_kernel.cuh -- the sm_100a kernel of the BF16 NT GEMM (DeepGEMM pages:
+// page 3 "核心功能" -- FP8, FP4 and BF16 GEMMs in the same dense and
+// m-grouped layouts).
+//
+//   D[m,n] = sum_k A[m,k] * B[n,k]     (A [M,K], B [N,K] BF16, K-major; D BF16)
+//
+// No block scales, so nothing is promoted on CUDA cores: the tensor cores
+// accumulate the whole K range in one FP32 TMEM accumulator per tile.  The
+// kernel is persistent and warp-specialised over the same tile scheduler as
+// the FP8 kernel (TileMap: dense raster, contiguous group lookup, masked tile
+// list built on the device):
+//
+//   warp 0      producer: one thread issues TMA loads of the A tile (128 rows)
+//               and the B tile (kBN rows) per 64-element K-block (128 bytes,
+//               128B swizzle -- the same shared-memory tiling as the FP8 path).
+//   warp 1      TMEM allocator + MMA issuer: 4 x tcgen05.mma.kind::f16 (K=16)
+//               per K-block into the tile's accumulator; two accumulators in
+//               rotation so the next tile's MMAs overlap this tile's epilogue.
+//   warps 4..7  epilogue: tcgen05.ld of the accumulator in 32-column chunks,
+//               BF16 round-to-nearest-even, 16-byte stores of each row.
+//
+// Every wait is bounded (BoundedWait): on timeout the kernel records
+// DG_ERR_TIMEOUT in the device status word and winds down instead of hanging.
+#pragma once
+
+#include "gemm_kernel.cuh"
+
+namespace dg {
+
+constexpr int kBf16Threads = 256;
+constexpr int kBf16BlockK = 64;          // BF16 elements per 128-byte K-block
+
+// Instruction descriptor, kind::f16: D = F32, A = B = BF16, both K-major.
+__host__ __device__ constexpr uint32_t bf16_idesc(int m, int n) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(n >> 3) << 17) |
+           (static_cast<uint32_t>(m >> 4) << 24);
+}
+
+template <int kBN, int kStages>
+struct Bf16Smem {
+    static constexpr int kXBytes = kTileX * 128;        // 128 rows x 64 BF16
+    static constexpr int kYBytes = kBN * 128;
+    static constexpr int kStageBytes = kXBytes + kYBytes;
+    static constexpr int kAccBufs = 2;
+    static constexpr int kBarOffset = kStages * kStageBytes;
+    static constexpr int kNumBars = 2 * kStages + 2 * kAccBufs + 1;
+    static constexpr int kMiscOffset = kBarOffset + kNumBars * 8;   // tmem addr, abort flag
+    static constexpr int kPrefixOffset = (kMiscOffset + 16 + 15) / 16 * 16;
+    static constexpr int kPrefixBytes = (kMaxGroups + 1) * 4;
+    static constexpr int kUsed = kPrefixOffset + kPrefixBytes;
+    static constexpr int kAlloc = (kUsed + 1024 > kMinSmem) ? kUsed + 1024 : kMinSmem;
+    static constexpr int kTmemCols = kAccBufs * kBN <= 256 ? 256 : 512;
+    static_assert(kAccBufs * kBN <= 512, "TMEM holds 512 columns");
+    static_assert(kStageBytes % 1024 == 0, "stage must keep 1024-byte alignment");
+    static_assert(kAlloc <= 227 * 1024, "shared memory budget");
+};
+
+template <int kBN, int kStages, int kLayout>
+__global__ void __launch_bounds__(kBf16Threads, 1)
+bf16_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
+                 const Params p) {
+    using L = Bf16Smem<kBN, kStages>;
+    using TM = TileMap<kBN, false, kLayout, 1>;
+    static_assert(kBN == 128 || kBN == 224 || kBN == 256, "tile N");
+    static_assert(kLayout != kKGrouped, "BF16: dense, contiguous and masked layouts");
+    constexpr int kAccBufs = L::kAccBufs;
+    constexpr int kEpiWarp0 = 4;
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    const uint32_t s_base = ptx::smem_u32(smem);
+    const uint32_t bar_base = s_base + L::kBarOffset;
+    auto full_bar = [&](int s) { return bar_base + 8u * s; };
+    auto empty_bar = [&](int s) { return bar_base + 8u * (kStages + s); };
+    auto tfull_bar = [&](int b) { return bar_base + 8u * (2 * kStages + b); };
+    auto tempty_bar = [&](int b) { return bar_base + 8u * (2 * kStages + kAccBufs + b); };
+    const uint32_t mma_done_bar = bar_base + 8u * (2 * kStages + 2 * kAccBufs);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kMiscOffset);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kMiscOffset + 4);
+    int *prefix = reinterpret_cast<int *>(smem + L::kPrefixOffset);
+
+    const int warp = threadIdx.x / 32;
+    const int lane = threadIdx.x % 32;
+    const BoundedWait wait{abort_flag, p.status, p.timeout_cycles};
+
+    if (threadIdx.x == 0) {
+        ptx::prefetch_tmap(&tm_a);
+        ptx::prefetch_tmap(&tm_b);
+        for (int i = 0; i < kStages; ++i) {
+            ptx::mbar_init(full_bar(i), 1);
+            ptx::mbar_init(empty_bar(i), 1);
+        }
+        for (int b = 0; b < kAccBufs; ++b) {
+            ptx::mbar_init(tfull_bar(b), 1);
+            ptx::mbar_init(tempty_bar(b), 4);          // one arrival per epilogue warp
+        }
+        ptx::mbar_init(mma_done_bar, 1);
+        *abort_flag = 0;
+        ptx::fence_mbar_init();
+    }
+    if (kLayout == kMasked && warp == kEpiWarp0) {
+        // exclusive prefix of tiles per group: ceil(masked_m[g] / 128) * weight blocks
+        const int nw = (p.N + TM::kWRows - 1) / TM::kWRows;
+        int carry = 0;
+        for (int base = 0; base < p.G; base += 32) {
+            const int g = base + lane;
+            int tiles = 0;
+            if (g < p.G) {
+                int mm = __ldg(p.masked_m + g);
+                if (mm < 0 || mm > p.M) {
+                    record_status(p.status, kStatusInvalid, kSiteBadMask);
+                    mm = mm < 0 ? 0 : p.M;
+                }
+                tiles = (mm + TM::kTokRows - 1) / TM::kTokRows * nw;
+            }
+            int incl = tiles;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int v = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += v;
+            }
+            if (g < p.G) prefix[g] = carry + incl - tiles;
+            carry += __shfl_sync(0xffffffffu, incl, 31);
+        }
+        if (lane == 0) prefix[p.G] = carry;
+    }
+    if (warp == 1) {
+        ptx::tmem_alloc(ptx::smem_u32(tmem_slot), L::kTmemCols);
+        ptx::tmem_relinquish();
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    const int num_tiles = TM::count(p, prefix);
+    const int t_first = static_cast<int>(blockIdx.x);
+    const int t_step = static_cast<int>(gridDim.x);
+    const int num_kb = p.num_kb;
+
+    if (warp == 0) {
+        // ============================================================ producer
+        __syncwarp();
+        if (ptx::elect_one()) {
+            int stage = 0;
+            uint32_t phase = 0;
+            long long issued = 0;
+            bool ok = (p.debug_flags & kDebugProducerIdle) == 0;
+            for (int t = t_first; ok && t < num_tiles; t += t_step) {
+                Tile tl;
+                if (!TM::decode(t, p, prefix, tl)) {
+                    if (kLayout == kContiguous && __ldg(p.m_indices + tl.tok0) >= p.G)
+                        record_status(p.status, kStatusInvalid, kSiteBadGroup);
+                    continue;
+                }
+                for (int kb = 0; kb < num_kb; ++kb) {
+                    if (!wait(empty_bar(stage), phase ^ 1u, kSiteProducerEmpty)) { ok = false; break; }
+                    const uint32_t sx = s_base + stage * L::kStageBytes;
+                    ptx::mbar_arrive_expect_tx(full_bar(stage), L::kStageBytes);
+                    ptx::tma_load_3d(sx, &tm_a, full_bar(stage), kb * kBf16BlockK, tl.a_row, tl.a_grp);
+                    ptx::tma_load_3d(sx + L::kXBytes, &tm_b, full_bar(stage), kb * kBf16BlockK, tl.n0,
+                                     tl.b_grp);
+                    ++issued;
+                    if (++stage == kStages) { stage = 0; phase ^= 1u; }
+                }
+            }
+            // never leave with TMA writes into shared memory in flight
+            const long long first = issued > kStages ? issued - kStages : 0;
+            for (long long i = first; i < issued; ++i) {
+                const uint32_t bar = full_bar(static_cast<int>(i % kStages));
+                const uint32_t par = static_cast<uint32_t>((i / kStages) & 1);
+                const long long start = clock64();
+                while (!ptx::mbar_try_wait(bar, par)) {
+                    if (clock64() - start > p.timeout_cycles) {
+                        record_status(p.status, kStatusTimeout, kSiteTeardownLoads);
+                        break;
+                    }
+                }
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ============================================================ MMA issuer
+        if (ptx::elect_one()) {
+            int stage = 0, buf = 0;
+            uint32_t phase = 0, tphase = 0;
+            bool ok = true;
+            const uint32_t idesc = bf16_idesc(kTileX, kBN);
+            for (int t = t_first; ok && t < num_tiles; t += t_step) {
+                Tile tl;
+                if (!TM::decode(t, p, prefix, tl)) continue;
+                if (!wait(tempty_bar(buf), tphase ^ 1u, kSiteMmaTmemEmpty)) { ok = false; break; }
+                const uint32_t dtm = tmem_base + static_cast<uint32_t>(buf * kBN);
+                for (int kb = 0; kb < num_kb; ++kb) {
+                    if (!wait(full_bar(stage), phase, kSiteMmaFull)) { ok = false; break; }
+                    ptx::tc_fence_after();
+                    const uint32_t sx = s_base + stage * L::kStageBytes;
+                    const uint64_t dx = sw128_desc(sx);
+                    const uint64_t dy = sw128_desc(sx + L::kXBytes);
+#pragma unroll
+                    for (int k = 0; k < kBf16BlockK / 16; ++k)
+                        ptx::mma_f16(dtm, dx + 2u * k, dy + 2u * k, idesc, (kb > 0 || k > 0) ? 1u : 0u);
+                    ptx::mma_commit(empty_bar(stage));
+                    if (++stage == kStages) { stage = 0; phase ^= 1u; }
+                }
+                if (!ok) break;
+                ptx::mma_commit(tfull_bar(buf));
+                if (++buf == kAccBufs) { buf = 0; tphase ^= 1u; }
+            }
+            ptx::mma_commit(mma_done_bar);
+        }
+        __syncwarp();
+    } else if (warp >= kEpiWarp0) {
+        // ============================================================ epilogue
+        const int quarter = warp & 3;
+        const int lrow = quarter * 32 + lane;
+        int buf = 0;
+        uint32_t tphase = 0;
+        for (int t = t_first; t < num_tiles; t += t_step) {
+            Tile tl;
+            if (!TM::decode(t, p, prefix, tl)) continue;
+            if (!wait(tfull_bar(buf), tphase, kSitePromoFull)) break;
+            ptx::tc_fence_after();
+            const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
+                                   static_cast<uint32_t>(buf * kBN);
+            const int my_tok = tl.tok0 + lrow;
+            const bool row_ok = my_tok < tl.tok_end;
+            const size_t row_base = kLayout == kMasked ? static_cast<size_t>(tl.g) * p.M : 0;
+            __nv_bfloat16 *drow = p.d + (row_base + my_tok) * static_cast<size_t>(p.N);
+#pragma unroll 1
+            for (int c = 0; c < kBN / 32; ++c) {
+                float v[32];
+                ptx::tmem_ld32p(taddr + c * 32, v);
+                ptx::tmem_wait_ld();
+                if (row_ok) {
+#pragma unroll
+                    for (int j = 0; j < 32; j += 8) {
+                        const int col = tl.n0 + c * 32 + j;
+                        if (col < p.N) {
+                            uint4 pk;
+                            __nv_bfloat162 h0 = __floats2bfloat162_rn(v[j + 0], v[j + 1]);
+                            __nv_bfloat162 h1 = __floats2bfloat162_rn(v[j + 2], v[j + 3]);
+                            __nv_bfloat162 h2 = __floats2bfloat162_rn(v[j + 4], v[j + 5]);
+                            __nv_bfloat162 h3 = __floats2bfloat162_rn(v[j + 6], v[j + 7]);
+                            pk.x = *reinterpret_cast<uint32_t *>(&h0);
+                            pk.y = *reinterpret_cast<uint32_t *>(&h1);
+                            pk.z = *reinterpret_cast<uint32_t *>(&h2);
+                            pk.w = *reinterpret_cast<uint32_t *>(&h3);
+                            *reinterpret_cast<uint4 *>(drow + col) = pk;
+                        }
+                    }
+                }
+            }
+            // the accumulator is free for the MMA warp's next tile
+            ptx::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(tempty_bar(buf));
+            if (++buf == kAccBufs) { buf = 0; tphase ^= 1u; }
+        }
+    }
+
+    // ---------------------------------------------------------------- teardown
+    if (warp == 1 && ptx::elect_one()) {
+        const long long start = clock64();
+        while (!ptx::mbar_try_wait(mma_done_bar, 0)) {
+            if (clock64() - start > p.timeout_cycles) {
+                record_status(p.status, kStatusTimeout, kSiteTeardownMma);
+                break;
+            }
+        }
+    }
+    __syncwarp();
+    ptx::tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc(tmem_base, L::kTmemCols);
+    }
+}
+
+}  // namespace dg

@@ -102,23 +102,28 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// 3-D uint8 tensor {K, rows, groups} (K innermost), box {128, box_rows, 1},
-// 128-byte swizzle, zero fill out of bounds.
-dg_status_t make_map(CUtensorMap *m, const void *base, long long K, long long rows,
-                     long long groups, int box_rows) {
+}  // namespace
+
+namespace dg_host {
+
+dg_status_t make_kmajor_map(CUtensorMap *m, const void *base, int elem_bytes, long long K,
+                            long long rows, long long groups, int box_rows) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) {
         std::snprintf(t_last_cuda_error, sizeof(t_last_cuda_error),
                       "cuTensorMapEncodeTiled entry point unavailable");
         return DG_ERR_CUDA;
     }
+    const cuuint64_t eb = static_cast<cuuint64_t>(elem_bytes);
     cuuint64_t dims[3] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows),
                           static_cast<cuuint64_t>(groups)};
-    cuuint64_t strides[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(K * rows)};
-    cuuint32_t box[3] = {static_cast<cuuint32_t>(dg::kBlockK), static_cast<cuuint32_t>(box_rows), 1};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(K) * eb, static_cast<cuuint64_t>(K * rows) * eb};
+    cuuint32_t box[3] = {static_cast<cuuint32_t>(128 / elem_bytes), static_cast<cuuint32_t>(box_rows), 1};
     cuuint32_t estr[3] = {1, 1, 1};
-    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(base), dims, strides,
-                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+    const CUtensorMapDataType dt = elem_bytes == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                                   : CU_TENSOR_MAP_DATA_TYPE_UINT8;
+    CUresult r = fn(m, dt, 3, const_cast<void *>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) {
         std::snprintf(t_last_cuda_error, sizeof(t_last_cuda_error),
@@ -126,6 +131,27 @@ dg_status_t make_map(CUtensorMap *m, const void *base, long long K, long long ro
         return DG_ERR_CUDA;
     }
     return DG_SUCCESS;
+}
+
+long long timeout_cycles() {
+    static long long v = [] {
+        const char *s = std::getenv("DG_WAIT_TIMEOUT_CYCLES");
+        long long x = s ? std::atoll(s) : 0;
+        return x > 0 ? x : (1LL << 32);   // ~2 s at 2 GHz; legitimate waits are micro- to milliseconds
+    }();
+    return v;
+}
+
+}  // namespace dg_host
+
+namespace {
+using namespace dg_host;
+
+// 3-D uint8 tensor {K, rows, groups} (K innermost), box {128, box_rows, 1},
+// 128-byte swizzle, zero fill out of bounds.
+dg_status_t make_map(CUtensorMap *m, const void *base, long long K, long long rows,
+                     long long groups, int box_rows) {
+    return make_kmajor_map(m, base, 1, K, rows, groups, box_rows);
 }
 
 // ------------------------------------------------------------------ validation
@@ -141,15 +167,6 @@ dg_status_t check_common(const void *a, const float *sfa, int ld_sfa, const void
     // TMA coordinates and element offsets stay within 32-bit ranges
     if (static_cast<long long>(K) > (1LL << 30) || N > (1 << 30)) return DG_ERR_UNSUPPORTED_SHAPE;
     return DG_SUCCESS;
-}
-
-long long timeout_cycles() {
-    static long long v = [] {
-        const char *s = std::getenv("DG_WAIT_TIMEOUT_CYCLES");
-        long long x = s ? std::atoll(s) : 0;
-        return x > 0 ? x : (1LL << 32);   // ~2 s at 2 GHz; legitimate waits are micro- to milliseconds
-    }();
-    return v;
 }
 
 // ------------------------------------------------------------------ launch

@@ -187,6 +187,17 @@ __device__ __forceinline__ void mma_f8f6f4(uint32_t d_tmem, uint64_t a_desc, uin
         : "memory");
 }
 
+// BF16 / FP16 MMA (kind::f16): D[tmem] (+)= A[smem] * B[smem]^T, FP32 accumulate.
+__device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                        uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
 // CTA-pair MMA (issued by one thread of the even CTA): A rows 0..M/2-1 come
 // from this CTA's smem and M/2..M-1 from the peer's (same offset), B is split
 // the same way along N; each CTA's TMEM receives its own M/2 rows.
