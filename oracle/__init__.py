@@ -13,6 +13,8 @@ Definition (DeepGEMM pages, page 2 "技术特性" and page 3 "核心功能"):
 BF16 GEMM (page 3 "核心功能"): D = sum_k A[m,k] * B[n,k], no block scales.
 K-grouped (page 3 "核心功能", k_grouped_gemm): group g sums only over its own
 ks[g] consecutive K columns, D[g] = the same sum over those K-blocks.
+Fused expert FFN (page 5 "03", Mega MoE without its communication): GEMM1 ->
+SwiGLU (FP64, rounded to FP32) -> per-token 1x128 quantiser -> GEMM2.
 Quantiser (page 2 "技术特性", dynamic fine-grained scaling): per row and
 128-wide K-block, s = amax / 448 in FP32, q = E4M3_RNE(clamp(x / s, +-448)).
 Every function is pinned (tests/test_oracle.py, tests/test_oracle_quant.py,
@@ -160,6 +162,40 @@ def gemm_bf16(layout: str, a_bits, b_bits, M, N, K, G=1, m_indices=None, masked_
     if rc:
         raise ValueError(f"oracle_bf16_gemm_nt rejected the input (rc={rc})")
     return d
+
+
+def silu(x: np.ndarray) -> np.ndarray:
+    """x * sigmoid(x) = x / (1 + exp(-x)), float64."""
+    with np.errstate(over="ignore"):
+        return x / (1.0 + np.exp(-x))
+
+
+def ffn_rows(prob, rows) -> dict:
+    """Fused expert FFN (contiguous layout) for the given valid rows:
+    h = block-scaled GEMM1 (FP64), act = silu(gate) * up in FP64, rounded to
+    FP32, quantised per 128 columns (s = amax/448, E4M3 codes), y = block-scaled
+    GEMM2 of the codes.  Returns h, act (FP32), q, s ([IB, len(rows)]) and y."""
+    rows = np.asarray(rows)
+    I, H = prob.I, prob.H
+    out = {"h": np.empty((len(rows), 2 * I)), "act": np.empty((len(rows), I), np.float32),
+           "q": np.empty((len(rows), I), np.uint8), "s": np.empty((I // 128, len(rows)), np.float32),
+           "y": np.empty((len(rows), H))}
+    groups = prob.m_indices[rows]
+    assert (groups >= 0).all(), "padding rows have no FFN output"
+    for g in np.unique(groups):
+        sel = np.flatnonzero(groups == g)
+        r = rows[sel]
+        n = len(r)
+        ld = (n + 3) // 4 * 4
+        sfa = np.zeros((H // 128, ld), np.float32)
+        sfa[:, :n] = prob.sfa[:, r]
+        h = gemm_dense(prob.a[r], sfa, ld, prob.w1[g], prob.sfb1[g], n, 2 * I, H)
+        hb = h.reshape(n, I // 128, 2, 128)
+        act = (silu(hb[:, :, 0, :]) * hb[:, :, 1, :]).reshape(n, I).astype(np.float32)
+        q, s = quantize_1x128(act, ld_sfa=ld)
+        y = gemm_dense(q, s, ld, prob.w2[g], prob.sfb2[g], n, H, I)
+        out["h"][sel], out["act"][sel], out["q"][sel], out["s"][:, sel], out["y"][sel] = h, act, q, s[:, :n], y
+    return out
 
 
 _LAYOUT_CODE = {"dense": 0, "contiguous": 1, "masked": 2}

@@ -526,3 +526,88 @@ def make_bf16_workload(name: str, seed_offset: int = 0) -> BF16Problem:
         return make_bf16_contiguous(counts, w["N"], w["K"], seed + 1000, name=name)
     masked_m = rng.integers(0, w["Mmax"] + 1, size=w["G"]).astype(np.int32)
     return make_bf16_masked(masked_m, w["Mmax"], w["N"], w["K"], seed + 1000, name=name)
+
+
+# ----------------------------------------------------------------------------- fused expert FFN inputs
+@dataclasses.dataclass
+class FFNProblem:
+    """Single-GPU expert FFN in the contiguous layout: tokens a [M_total, H]
+    (E4M3, 1x128 scales), w1 [G, 2I, H] with gate and up rows interleaved per
+    128 rows (block 2j = gate rows 128j.., block 2j+1 = the matching up rows),
+    w2 [G, H, I]; both weights with 128x128 scales."""
+    M: int                     # M_total (groups padded to 128 rows)
+    H: int
+    I: int
+    G: int
+    a: np.ndarray
+    sfa: np.ndarray
+    ld_sfa: int
+    w1: np.ndarray
+    sfb1: np.ndarray
+    w2: np.ndarray
+    sfb2: np.ndarray
+    m_indices: np.ndarray
+    name: str = ""
+    layout: str = "ffn_contiguous"
+
+    def valid_rows(self) -> int:
+        return int((self.m_indices >= 0).sum())
+
+    def groups_touched(self) -> int:
+        return int(len(np.unique(self.m_indices[self.m_indices >= 0])))
+
+    def flops(self) -> float:
+        """Both GEMMs: 2 * rows * (2I * H + H * I)."""
+        return 2.0 * self.valid_rows() * (2 * self.I * self.H + self.H * self.I)
+
+    def bytes(self) -> float:
+        """A, the touched experts' weights, the intermediate codes (written and
+        read) with their scales, and y."""
+        r, g = self.valid_rows(), self.groups_touched()
+        kb, ib = self.H // BLOCK, self.I // BLOCK
+        return float(r * self.H + r * kb * 4 + g * 3 * self.I * self.H
+                     + g * (2 * ib * kb + kb * ib) * 4 + 2 * (r * self.I + r * ib * 4) + 2 * r * self.H)
+
+
+def make_ffn_contiguous(counts, H: int, I: int, seed: int, name: str = "") -> FFNProblem:
+    """Token rows as the contiguous GEMM's A (N(0,1), 1x128 scales, padding rows
+    NaN); weights N(0,1)/sqrt(fan-in) quantised per 128x128 block; gate and up
+    interleaved per 128 rows in w1."""
+    assert H % BLOCK == 0 and I % BLOCK == 0
+    base = make_contiguous(counts, 2 * I, H, seed, name=name)     # a, sfa, m_indices (w unused)
+    rng = np.random.default_rng(seed + 500)
+    G = len(counts)
+    gate = _normal(rng, (G, I, H)) / np.float32(np.sqrt(H))
+    up = _normal(rng, (G, I, H)) / np.float32(np.sqrt(H))
+    down = _normal(rng, (G, H, I)) / np.float32(np.sqrt(I))
+    w1_32 = np.empty((G, 2 * I, H), np.float32)
+    for j in range(I // BLOCK):
+        w1_32[:, 2 * j * BLOCK:(2 * j + 1) * BLOCK] = gate[:, j * BLOCK:(j + 1) * BLOCK]
+        w1_32[:, (2 * j + 1) * BLOCK:(2 * j + 2) * BLOCK] = up[:, j * BLOCK:(j + 1) * BLOCK]
+    w1 = np.empty((G, 2 * I, H), np.uint8)
+    sfb1 = np.empty((G, 2 * I // BLOCK, H // BLOCK), np.float32)
+    w2 = np.empty((G, H, I), np.uint8)
+    sfb2 = np.empty((G, H // BLOCK, I // BLOCK), np.float32)
+    for g in range(G):
+        w1[g], sfb1[g] = quantize_blocks_128x128(w1_32[g])
+        w2[g], sfb2[g] = quantize_blocks_128x128(down[g])
+    return FFNProblem(base.M, H, I, G, base.a, base.sfa, base.ld_sfa, w1, sfb1, w2, sfb2,
+                      base.m_indices, name=name)
+
+
+def make_ffn_multinomial(G: int, tokens: int, H: int, I: int, seed: int, name: str = "") -> FFNProblem:
+    rng = np.random.default_rng(seed)
+    counts = rng.multinomial(tokens, [1.0 / G] * G)
+    return make_ffn_contiguous(counts, H, I, seed + 1000, name=name)
+
+
+# an expert FFN of a DeepSeek-V3-sized MoE layer on 4 experts: hidden 7168,
+# intermediate 2048, 32768 routed tokens (the contiguous workload's tokens)
+FFN_WORKLOADS = {
+    "ffn_g4": dict(G=4, tokens=32768, H=7168, I=2048, seed=15),
+}
+
+
+def make_ffn_workload(name: str, seed_offset: int = 0) -> FFNProblem:
+    w = dict(FFN_WORKLOADS[name])
+    return make_ffn_multinomial(w["G"], w["tokens"], w["H"], w["I"], w["seed"] + seed_offset, name=name)
