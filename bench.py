@@ -40,7 +40,7 @@ UNIT = {"dense_tiny": "TFLOP/s", "dense_decode_m64": "GB/s", "dense_decode_m128"
         "dense_large": "TFLOP/s", "contiguous_g4": "TFLOP/s", "masked_g16": "GB/s",
         "kgrouped_g4": "TFLOP/s",
         "bf16_dense_large": "TFLOP/s", "bf16_contiguous_g4": "TFLOP/s", "bf16_masked_g16": "GB/s",
-        "bf16_dense_decode_m64": "GB/s",
+        "bf16_dense_decode_m64": "GB/s", "ffn_g4": "TFLOP/s",
         "quant_tiny": "GB/s", "quant_tokens_32768": "GB/s", "quant_masked_g16": "GB/s"}
 # the kernel each workload times, and the sources whose hash keys its ncu summary
 KERNEL_SOURCES = {
@@ -172,6 +172,8 @@ def rank_problem(workload: str, rank: int):
         return W.make_quant_workload(workload, seed_offset=7919 * rank)
     if is_bf16(workload):
         return W.make_bf16_workload(workload, seed_offset=7919 * rank)
+    if workload in W.FFN_WORKLOADS:
+        return W.make_ffn_workload(workload, seed_offset=7919 * rank)
     if rank == 0:
         return W.make_workload(workload)
     spec = dict(W.WORKLOADS[workload])
@@ -270,6 +272,34 @@ class Bf16Call:
         return self.d.numel() * self.d.element_size()
 
 
+class FFNCall:
+    """Pinned tokens and expert weights, device intermediate and output, and the
+    fused expert FFN call (two launches: GEMM1 + SwiGLU + requantisation, GEMM2)."""
+
+    def __init__(self, prob, dev):
+        import numpy as np
+        import torch
+        self.prob = prob
+        t = lambda x: torch.from_numpy(np.ascontiguousarray(x)).pin_memory()
+        self.host = {"a": t(prob.a), "sfa": t(prob.sfa), "w1": t(prob.w1), "sfb1": t(prob.sfb1),
+                     "w2": t(prob.w2), "sfb2": t(prob.sfb2), "m_indices": t(prob.m_indices)}
+        self.q = torch.empty((prob.M, prob.I), dtype=torch.uint8, device=dev)
+        self.s = torch.empty((prob.I // 128, prob.ld_sfa), dtype=torch.float32, device=dev)
+        self.y = torch.empty((prob.M, prob.H), dtype=torch.bfloat16, device=dev)
+        self.y_host = torch.empty((prob.M, prob.H), dtype=torch.bfloat16).pin_memory()
+
+    def call(self, t, stream):
+        import moe_grouped_gemm_fp32_b200 as dg
+        dg.dg_m_grouped_fp8_ffn_contiguous(t["a"], t["sfa"], t["w1"], t["sfb1"], t["w2"], t["sfb2"],
+                                           self.q, self.s, self.y, t["m_indices"], stream)
+
+    def read_back(self):
+        self.y_host.copy_(self.y, non_blocking=True)
+
+    def d2h_bytes(self) -> int:
+        return self.y.numel() * self.y.element_size()
+
+
 class QuantCall:
     """Pinned BF16 activations, device codes and scales, and the quantiser call."""
 
@@ -311,7 +341,8 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.set_device(dev)
     prob = rank_problem(args.workload, rank)
 
-    op = (QuantCall if is_quant(args.workload) else Bf16Call if is_bf16(args.workload) else GemmCall)(prob, dev)
+    op = (QuantCall if is_quant(args.workload) else Bf16Call if is_bf16(args.workload)
+          else FFNCall if prob.layout == "ffn_contiguous" else GemmCall)(prob, dev)
     host = op.host
     devt = {k: v.to(dev, non_blocking=False) for k, v in host.items()}
     flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
@@ -460,6 +491,22 @@ def cpu_baseline(prob, unit, budget_s=10.0):
         return quant_cpu_baseline(prob, budget_s)
     if not hasattr(prob, "sfa"):
         return bf16_cpu_baseline(prob, unit, budget_s)
+    if prob.layout == "ffn_contiguous":
+        oracle.build()
+        valid = np.flatnonzero(prob.m_indices >= 0)
+        t0 = time.perf_counter()
+        oracle.ffn_rows(prob, valid[:: max(1, len(valid) // 8)][:8])
+        per_row = (time.perf_counter() - t0) / 8
+        n = max(8, min(len(valid), int(budget_s / per_row)))
+        pick = valid[:: max(1, len(valid) // n)][:n]
+        t0 = time.perf_counter()
+        oracle.ffn_rows(prob, pick)
+        dt = time.perf_counter() - t0
+        secs = dt * len(valid) / len(pick)
+        return {"value": prob.flops() / secs / 1e12, "unit": unit, "cores": len(os.sched_getaffinity(0)),
+                "kind": "oracle", "seconds_per_step": secs,
+                "sample": f"{len(pick)} of {len(valid)} token rows through both GEMMs, {dt:.1f} s, "
+                          f"scaled linearly to the whole workload"}
     oracle.build()
     cores = len(os.sched_getaffinity(0))
     t0 = time.perf_counter()
@@ -557,6 +604,9 @@ def run_reference(args, rank, world):
 
 
 def shape_config(prob):
+    if getattr(prob, "layout", "") == "ffn_contiguous":
+        return {"layout": "contiguous expert FFN (GEMM1 + SwiGLU + requantise, GEMM2)", "G": prob.G,
+                "M_total": prob.M, "valid_rows": prob.valid_rows(), "H": prob.H, "I": prob.I}
     if hasattr(prob, "flops") and not hasattr(prob, "sfa"):   # BF16 GEMM
         c = {"layout": prob.layout, "N": prob.N, "K": prob.K, "operands": "bf16"}
         if prob.layout == "dense":

@@ -136,6 +136,49 @@ DG_API dg_status_t dg_k_grouped_fp8_gemm_nt_contiguous(const uint8_t *a, const f
                                                        int K, void *stream);
 
 /*
+ * Fused expert FFN, first stage (page 5 "03" -- Mega MoE fuses the first
+ * layer's GEMM, the SwiGLU activation and the second layer into one MoE
+ * kernel; here on one GPU, without the expert-parallel dispatch and combine):
+ * the contiguous M-grouped FP8 GEMM of the gate and up projections, whose
+ * epilogue applies SwiGLU and re-quantises the activation per token and
+ * 128-column block, writing the second GEMM's A operand directly (the FP32
+ * accumulators never go to memory).
+ *   a, sfa, m_indices: as for dg_m_grouped_fp8_gemm_nt_contiguous (K = hidden size)
+ *   b   [G, N, K] E4M3, N = 2 * I: for each 128-column block j of the
+ *       intermediate size I, weight rows [256 j, 256 j + 128) are the gate
+ *       projection and rows [256 j + 128, 256 j + 256) the up projection
+ *       ("interleaved by 128"); sfb [G, N/128, K/128] FP32.
+ *   With h = the promoted FP32 product (as in the GEMMs above):
+ *     act[m, 128 j + c] = silu(h[m, 256 j + c]) * h[m, 256 j + 128 + c],
+ *     silu(x) = x / (1 + exp(-x)), in FP32;
+ *     per row and 128-column block: s = amax / 448 (1 if amax == 0),
+ *     q = E4M3_RNE(act / s) (IEEE quotient; values saturate at +-448).
+ *   q_out [M_total, I] E4M3; s_out [I/128, ld_s_out] FP32 (MN-major,
+ *       ld_s_out >= M_total, a multiple of 4).  Rows of 128-row blocks whose
+ *       first row is padding are not written; padding rows inside a block may be.
+ * M_total % 128 == 0, N % 256 == 0.
+ */
+DG_API dg_status_t dg_m_grouped_fp8_gemm_swiglu_quant_contiguous(
+    const uint8_t *a, const float *sfa, int ld_sfa, const uint8_t *b, const float *sfb,
+    uint8_t *q_out, float *s_out, int ld_s_out, const int32_t *m_indices, int M_total, int N, int K,
+    int G, void *stream);
+
+/*
+ * Fused expert FFN on one GPU: the first stage above, then the contiguous
+ * M-grouped FP8 GEMM of the down projection on its output:
+ *   y = dg_m_grouped_fp8_gemm_nt_contiguous(q_mid, s_mid, w2 [G, H, I], sfb2 [G, H/128, I/128])
+ * a [M_total, H] E4M3 with sfa; w1 [G, 2I, H] (interleaved by 128) with sfb1;
+ * q_mid [M_total, I] and s_mid [I/128, ld_mid] are caller-owned intermediate
+ * buffers; y [M_total, H] BF16.  Two launches on the stream, no host sync.
+ */
+DG_API dg_status_t dg_m_grouped_fp8_ffn_contiguous(const uint8_t *a, const float *sfa, int ld_sfa,
+                                                   const uint8_t *w1, const float *sfb1,
+                                                   const uint8_t *w2, const float *sfb2,
+                                                   uint8_t *q_mid, float *s_mid, int ld_mid, void *y,
+                                                   const int32_t *m_indices, int M_total, int H,
+                                                   int I, int G, void *stream);
+
+/*
  * BF16 GEMMs (page 3 "核心功能": FP8, FP4 and BF16 GEMM operations, in the same
  * dense and m-grouped layouts):
  *   D[m,n] = sum_k A[m,k] * B[n,k]    accumulated in FP32, stored as BF16 (RNE)

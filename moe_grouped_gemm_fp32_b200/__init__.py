@@ -59,6 +59,8 @@ def lib() -> ctypes.CDLL:
     L.dg_m_grouped_fp8_gemm_nt_contiguous.argtypes = [P, P, I, P, P, P, P, I, I, I, I, P]
     L.dg_m_grouped_fp8_gemm_nt_masked.argtypes = [P, P, I, P, P, P, P, I, I, I, I, P]
     L.dg_k_grouped_fp8_gemm_nt_contiguous.argtypes = [P, P, I, P, P, P, P, I, I, I, I, P]
+    L.dg_m_grouped_fp8_gemm_swiglu_quant_contiguous.argtypes = [P, P, I, P, P, P, P, I, P, I, I, I, I, P]
+    L.dg_m_grouped_fp8_ffn_contiguous.argtypes = [P, P, I, P, P, P, P, P, P, I, P, P, I, I, I, I, P]
     L.dg_bf16_gemm_nt.argtypes = [P, P, P, I, I, I, P]
     L.dg_m_grouped_bf16_gemm_nt_contiguous.argtypes = [P, P, P, P, I, I, I, I, P]
     L.dg_m_grouped_bf16_gemm_nt_masked.argtypes = [P, P, P, P, I, I, I, I, P]
@@ -66,6 +68,7 @@ def lib() -> ctypes.CDLL:
     L.dg_per_token_cast_to_fp8_masked.argtypes = [P, P, P, I, P, I, I, I, P]
     for f in ("dg_fp8_gemm_nt", "dg_m_grouped_fp8_gemm_nt_contiguous",
               "dg_m_grouped_fp8_gemm_nt_masked", "dg_k_grouped_fp8_gemm_nt_contiguous",
+              "dg_m_grouped_fp8_gemm_swiglu_quant_contiguous", "dg_m_grouped_fp8_ffn_contiguous",
               "dg_bf16_gemm_nt", "dg_m_grouped_bf16_gemm_nt_contiguous",
               "dg_m_grouped_bf16_gemm_nt_masked",
               "dg_per_token_cast_to_fp8",
@@ -180,6 +183,41 @@ def dg_k_grouped_fp8_gemm_nt_contiguous(a, sfa, b, sfb, d, ks, stream=None):
     _check(st, "dg_k_grouped_fp8_gemm_nt_contiguous")
     return d
 
+
+
+# --------------------------------------------------------------------------- fused expert FFN
+def dg_m_grouped_fp8_gemm_swiglu_quant_contiguous(a, sfa, b, sfb, q_out, s_out, m_indices, stream=None):
+    """First FFN stage: contiguous FP8 GEMM with gate/up weights b [G, 2I, K]
+    (interleaved per 128 rows) whose epilogue writes E4M3 codes q_out
+    [M_total, I] and scales s_out [I/128, ld] of silu(gate) * up."""
+    import torch
+    M_total, K = a.shape
+    G, N, _ = b.shape
+    st = lib().dg_m_grouped_fp8_gemm_swiglu_quant_contiguous(
+        _req(a, torch.uint8, "a", 2), _req(sfa, torch.float32, "sfa", 2), sfa.shape[-1],
+        _req(b, torch.uint8, "b", 3), _req(sfb, torch.float32, "sfb", 3),
+        _req(q_out, torch.uint8, "q_out", 2), _req(s_out, torch.float32, "s_out", 2), s_out.shape[-1],
+        _req(m_indices, torch.int32, "m_indices", 1), M_total, N, K, G, _stream_handle(stream))
+    _check(st, "dg_m_grouped_fp8_gemm_swiglu_quant_contiguous")
+    return q_out, s_out
+
+
+def dg_m_grouped_fp8_ffn_contiguous(a, sfa, w1, sfb1, w2, sfb2, q_mid, s_mid, y, m_indices, stream=None):
+    """Fused expert FFN on one GPU: y [M_total, H] (bfloat16) from tokens a
+    [M_total, H], w1 [G, 2I, H] (gate/up interleaved per 128 rows), w2 [G, H, I];
+    q_mid [M_total, I] / s_mid [I/128, ld] are the caller's intermediate buffers."""
+    import torch
+    M_total, H = a.shape
+    G, I2, _ = w1.shape
+    st = lib().dg_m_grouped_fp8_ffn_contiguous(
+        _req(a, torch.uint8, "a", 2), _req(sfa, torch.float32, "sfa", 2), sfa.shape[-1],
+        _req(w1, torch.uint8, "w1", 3), _req(sfb1, torch.float32, "sfb1", 3),
+        _req(w2, torch.uint8, "w2", 3), _req(sfb2, torch.float32, "sfb2", 3),
+        _req(q_mid, torch.uint8, "q_mid", 2), _req(s_mid, torch.float32, "s_mid", 2), s_mid.shape[-1],
+        _req(y, torch.bfloat16, "y", 2), _req(m_indices, torch.int32, "m_indices", 1),
+        M_total, H, I2 // 2, G, _stream_handle(stream))
+    _check(st, "dg_m_grouped_fp8_ffn_contiguous")
+    return y
 
 # --------------------------------------------------------------------------- BF16 GEMMs
 def dg_bf16_gemm_nt(a, b, d, stream=None):

@@ -170,11 +170,11 @@ dg_status_t check_common(const void *a, const float *sfa, int ld_sfa, const void
 }
 
 // ------------------------------------------------------------------ launch
-template <int kBN, bool kSwap, int kStages, int kLayout, int kCtaGroup = 1>
+template <int kBN, bool kSwap, int kStages, int kLayout, int kCtaGroup = 1, bool kSwiGLU = false>
 dg_status_t launch(const CUtensorMap &ma, const CUtensorMap &mb, const dg::Params &p, int grid_x,
                    int grid_y, int cluster_x, cudaStream_t stream) {
     using L = dg::SmemLayout<kBN, kSwap, kStages, kCtaGroup, kSwap && kLayout == dg::kDense && kBN <= 128>;
-    auto kernel = dg::fp8_gemm_kernel<kBN, kSwap, kStages, kLayout, kCtaGroup>;
+    auto kernel = dg::fp8_gemm_kernel<kBN, kSwap, kStages, kLayout, kCtaGroup, kSwiGLU>;
     static bool attr_done[kMaxDevices] = {};
     int dev = 0;
     cudaGetDevice(&dev);
@@ -507,6 +507,47 @@ dg_status_t dg_k_grouped_fp8_gemm_nt_contiguous(const uint8_t *a, const float *s
     if ((st = make_map(&mb, b, K, N, 1, bn / 2)) != DG_SUCCESS) return st;
     if (bn == 224) return launch<224, false, 6, dg::kKGrouped, 2>(ma, mb, p, 2 * pairs, 1, 2, s);
     return launch<256, false, 6, dg::kKGrouped, 2>(ma, mb, p, 2 * pairs, 1, 2, s);
+}
+
+dg_status_t dg_m_grouped_fp8_gemm_swiglu_quant_contiguous(
+    const uint8_t *a, const float *sfa, int ld_sfa, const uint8_t *b, const float *sfb,
+    uint8_t *q_out, float *s_out, int ld_s_out, const int32_t *m_indices, int M_total, int N, int K,
+    int G, void *stream) {
+    // d is not written in this mode; pass q_out to the common checks in its place
+    dg_status_t st = check_common(a, sfa, ld_sfa, b, sfb, q_out, M_total, N, K);
+    if (st != DG_SUCCESS) return st;
+    if (!m_indices || !s_out || G <= 0) return DG_ERR_INVALID_VALUE;
+    if (M_total % 128 != 0 || N % 256 != 0) return DG_ERR_UNSUPPORTED_SHAPE;
+    if (ld_s_out < M_total || ld_s_out <= 0) return DG_ERR_INVALID_VALUE;
+    if (ld_s_out % 4 != 0 || !aligned16(s_out)) return DG_ERR_MISALIGNED;
+    const DeviceInfo *info = nullptr;
+    if ((st = device_info(&info)) != DG_SUCCESS) return st;
+    if (M_total == 0) return DG_SUCCESS;
+    dg::Params p = base_params(sfa, ld_sfa, sfb, nullptr, M_total, N, K, G, info);
+    p.m_indices = m_indices;
+    p.q_out = q_out;
+    p.s_out = s_out;
+    p.ld_s_out = ld_s_out;
+    CUtensorMap ma, mb;
+    if ((st = make_map(&ma, a, K, M_total, 1, 128)) != DG_SUCCESS) return st;
+    if ((st = make_map(&mb, b, K, N, G, 256)) != DG_SUCCESS) return st;
+    const int tiles = (M_total / 128) * (N / 256);
+    const int grid = tiles < info->num_sms ? tiles : info->num_sms;
+    return launch<256, false, 4, dg::kContiguous, 1, true>(ma, mb, p, grid, 1, 1, static_cast<cudaStream_t>(stream));
+}
+
+dg_status_t dg_m_grouped_fp8_ffn_contiguous(const uint8_t *a, const float *sfa, int ld_sfa,
+                                            const uint8_t *w1, const float *sfb1, const uint8_t *w2,
+                                            const float *sfb2, uint8_t *q_mid, float *s_mid,
+                                            int ld_mid, void *y, const int32_t *m_indices,
+                                            int M_total, int H, int I, int G, void *stream) {
+    if (I <= 0 || I % 128 != 0) return DG_ERR_UNSUPPORTED_SHAPE;
+    if (!y) return DG_ERR_INVALID_VALUE;
+    dg_status_t st = dg_m_grouped_fp8_gemm_swiglu_quant_contiguous(a, sfa, ld_sfa, w1, sfb1, q_mid, s_mid, ld_mid,
+                                                                   m_indices, M_total, 2 * I, H, G, stream);
+    if (st != DG_SUCCESS) return st;
+    return dg_m_grouped_fp8_gemm_nt_contiguous(q_mid, s_mid, ld_mid, w2, sfb2, y, m_indices, M_total, H, I, G,
+                                               stream);
 }
 
 int dg_get_m_alignment_for_contiguous_layout(void) { return 128; }

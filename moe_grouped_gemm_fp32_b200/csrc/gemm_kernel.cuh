@@ -95,6 +95,11 @@ struct Params {
     int num_kb, num_nb;
     int split;  // CTAs per cluster along K (swap mode); 1 = persistent
     int debug_flags;
+    // SwiGLU-quantise epilogue (fused expert FFN, first GEMM): E4M3 codes
+    // [rows][N/2] and FP32 scales [N/256][ld_s_out] of silu(gate) * up
+    uint8_t *q_out;
+    float *s_out;
+    int ld_s_out;
 };
 
 constexpr int kDebugProducerIdle = 1;   // fault injection: the producer never loads
@@ -342,7 +347,8 @@ struct SmemLayout {
     // Each K-block's partial lives from its MMA until the promotion warps have
     // read it; more buffers let the MMAs run further ahead of the promotion.
     static constexpr int kAccBufs = 512 / kBN >= 4 ? 4 : (512 / kBN >= 3 ? 3 : 2);
-    static constexpr int kNumBars = 2 * kStages + 2 * kAccBufs + 1 + (kSwap ? 3 * kSlots : 0);
+    // + 2: the SwiGLU epilogue's amax-exchange barriers (one per tile parity)
+    static constexpr int kNumBars = 2 * kStages + 2 * kAccBufs + 1 + (kSwap ? 3 * kSlots : 0) + 2;
     static constexpr int kMiscOffset = kBarOffset + kNumBars * 8;     // tmem addr, abort flag
     static constexpr int kPrefixOffset = (kMiscOffset + 16 + 15) / 16 * 16;
     static constexpr int kPrefixBytes = (kMaxGroups + 1) * 4;
@@ -367,10 +373,15 @@ struct SmemLayout {
     static_assert(kAlloc <= 227 * 1024, "shared memory budget");
 };
 
-template <int kBN, bool kSwap, int kStages, int kLayout, int kCtaGroup>
+template <int kBN, bool kSwap, int kStages, int kLayout, int kCtaGroup, bool kSwiGLU = false>
 __global__ void __launch_bounds__(num_threads(kSwap), 1)
 fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                 const Params p) {
+    // SwiGLU epilogue: a 256-column tile is one 128-row gate block of the
+    // weights followed by the matching 128-row up block; each promotion
+    // warpgroup owns 64 gate columns and the 64 up columns they pair with
+    static_assert(!kSwiGLU || (kBN == 256 && !kSwap && kCtaGroup == 1 && kLayout == kContiguous),
+                  "SwiGLU epilogue: contiguous layout, 1-CTA 256-column tiles");
     // dense swap-mode kernels may run split-K (one tile per cluster)
     constexpr bool kSplitK = kSwap && kLayout == kDense && kBN <= 128;
     // the producer starts loading before the set-up barrier when nothing it
@@ -406,6 +417,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
     auto sfull_bar = [&](int i) { return bar_base + 8u * (2 * kStages + 2 * kAccBufs + 1 + i); };
     auto sready_bar = [&](int i) { return bar_base + 8u * (2 * kStages + 2 * kAccBufs + 1 + kSlots + i); };
     auto sempty_bar = [&](int i) { return bar_base + 8u * (2 * kStages + 2 * kAccBufs + 1 + 2 * kSlots + i); };
+    auto xchg_bar = [&](int i) { return bar_base + 8u * (L::kNumBars - 2 + i); };
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kMiscOffset);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kMiscOffset + 4);
     const uint32_t slot_base = s_base + L::kSlotOffset;
@@ -441,6 +453,8 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
             ptx::mbar_init(tempty_bar(b), 8 * kCtaGroup);   // every promotion warp of the pair
         }
         ptx::mbar_init(mma_done_bar, 1);
+        ptx::mbar_init(xchg_bar(0), 256);     // both promotion warpgroups
+        ptx::mbar_init(xchg_bar(1), 256);
         *abort_flag = 0;
         ptx::fence_mbar_init();
     }
@@ -803,6 +817,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
     };
     Tile last_tile{0, 0, 0, 0, 0, 0, 0, 3};
     bool have_tile = false;
+    int epi_parity = 0;   // SwiGLU epilogue: exchange-buffer parity
     int last_nvalid = 0;
     if (promo) {
         int stage = 0, buf = 0, sslot = 0;
@@ -883,7 +898,11 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
                         constexpr int kFull = 32;
                         const int ncol = (r + 1) * 32 <= kHalf ? kFull : kHalf - r * 32;   // 32 or 16
                         float v[32];
-                        const uint32_t ta = taddr + static_cast<uint32_t>(half * kHalf + r * 32);
+                        // this warpgroup's tile columns for round r (SwiGLU: two gate
+                        // rounds, then the two matching up rounds)
+                        const int rcol = kSwiGLU ? (r < 2 ? 64 * half + 32 * r : 128 + 64 * half + 32 * (r - 2))
+                                                 : half * kHalf + r * 32;
+                        const uint32_t ta = taddr + static_cast<uint32_t>(rcol);
                         if (ncol == 32) ptx::tmem_ld32p(ta, v);
                         else ptx::tmem_ld16p(ta, v);
                         ptx::tmem_wait_ld();
@@ -891,7 +910,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
 #pragma unroll
                         for (int q = 0; q < 4; ++q) {
                             if (q * 8 < ncol) {
-                                const int col = half * kHalf + r * 32 + q * 8;
+                                const int col = rcol + q * 8;
                                 const int blk = (tl.n0 + col) / 128 - wblk0;
                                 float sc = sblk[0];
 #pragma unroll
@@ -958,7 +977,50 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
             if (clustered) break;   // one tile; reduced below
             // ------------------------------------------------ epilogue (direct)
             const size_t row_base = (kLayout == kMasked || kLayout == kKGrouped) ? static_cast<size_t>(tl.g) * p.M : 0;
-            if (!kSwap) {
+            if constexpr (kSwiGLU) {
+                // act = silu(gate) * up for this thread's 64 columns of the tile's
+                // 128-column activation block; the block's amax is combined with
+                // the other warpgroup's through shared memory (one float per row,
+                // double-buffered by tile parity), then the 64 values are quantised
+                // like the per-token 1x128 quantiser: s = amax / 448, codes =
+                // E4M3_RNE(act / s) with the IEEE quotient.
+                float pmax = 0.f;
+#pragma unroll
+                for (int c = 0; c < 64; ++c) {
+                    const float g = acc[c];
+                    const float a = g / (1.0f + expf(-g)) * acc[64 + c];
+                    acc[c] = a;
+                    pmax = fmaxf(pmax, fabsf(a));
+                }
+                const int par = epi_parity & 1;
+                float *xbuf = reinterpret_cast<float *>(prefix) + par * 256;
+                xbuf[half * 128 + lrow] = pmax;
+                ptx::mbar_arrive(xchg_bar(par));          // release: the store above is visible
+                if (!wait(xchg_bar(par), static_cast<uint32_t>((epi_parity >> 1) & 1), kSitePromoFull)) break;
+                const float amax = fmaxf(pmax, xbuf[(half ^ 1) * 128 + lrow]);
+                ++epi_parity;
+                const float sc = amax == 0.0f ? 1.0f : __fdiv_rn(amax, 448.0f);
+                if (tok_ok) {
+                    const int ablk = tl.n0 / 256;                 // 128-column activation block
+                    const int ncols = p.N / 2;
+                    uint8_t *qrow = p.q_out + (row_base + my_tok) * static_cast<size_t>(ncols) + ablk * 128 + 64 * half;
+#pragma unroll
+                    for (int c = 0; c < 64; c += 16) {
+                        uint32_t w[4];
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            uint16_t lo, hi;
+                            const float t0 = __fdiv_rn(acc[c + 4 * j + 0], sc), t1 = __fdiv_rn(acc[c + 4 * j + 1], sc);
+                            const float t2 = __fdiv_rn(acc[c + 4 * j + 2], sc), t3 = __fdiv_rn(acc[c + 4 * j + 3], sc);
+                            asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(lo) : "f"(t1), "f"(t0));
+                            asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(hi) : "f"(t3), "f"(t2));
+                            w[j] = static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
+                        }
+                        *reinterpret_cast<uint4 *>(qrow + c) = make_uint4(w[0], w[1], w[2], w[3]);
+                    }
+                    if (half == 0) p.s_out[static_cast<size_t>(ablk) * p.ld_s_out + row_base + my_tok] = sc;
+                }
+            } else if (!kSwap) {
                 if (tok_ok) {
                     __nv_bfloat16 *drow = p.d + (row_base + my_tok) * static_cast<size_t>(p.N);
 #pragma unroll
