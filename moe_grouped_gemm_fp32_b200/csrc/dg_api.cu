@@ -147,6 +147,34 @@ long long timeout_cycles() {
 namespace {
 using namespace dg_host;
 
+// D as a 2-D BF16 tensor {N, rows} (masked / K-grouped: all groups' rows
+// stacked), box {32 columns, 32 rows} with 64-byte swizzle: the TMA-store
+// epilogue's box.  A null d (no BF16 output) gives an all-zero map the kernel
+// never uses.
+dg_status_t make_d_map(CUtensorMap *m, void *d, long long N, long long rows) {
+    std::memset(m, 0, sizeof(*m));
+    if (!d || rows <= 0) return DG_SUCCESS;
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) {
+        std::snprintf(t_last_cuda_error, sizeof(t_last_cuda_error),
+                      "cuTensorMapEncodeTiled entry point unavailable");
+        return DG_ERR_CUDA;
+    }
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(N) * 2};
+    cuuint32_t box[2] = {32, 32};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+                    CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        std::snprintf(t_last_cuda_error, sizeof(t_last_cuda_error),
+                      "cuTensorMapEncodeTiled (D) failed (CUresult %d)", static_cast<int>(r));
+        return DG_ERR_CUDA;
+    }
+    return DG_SUCCESS;
+}
+
 // 3-D uint8 tensor {K, rows, groups} (K innermost), box {128, box_rows, 1},
 // 128-byte swizzle, zero fill out of bounds.
 dg_status_t make_map(CUtensorMap *m, const void *base, long long K, long long rows,
@@ -171,8 +199,8 @@ dg_status_t check_common(const void *a, const float *sfa, int ld_sfa, const void
 
 // ------------------------------------------------------------------ launch
 template <int kBN, bool kSwap, int kStages, int kLayout, int kCtaGroup = 1, bool kSwiGLU = false>
-dg_status_t launch(const CUtensorMap &ma, const CUtensorMap &mb, const dg::Params &p, int grid_x,
-                   int grid_y, int cluster_x, cudaStream_t stream) {
+dg_status_t launch(const CUtensorMap &ma, const CUtensorMap &mb, const CUtensorMap &md, const dg::Params &p,
+                   int grid_x, int grid_y, int cluster_x, cudaStream_t stream) {
     using L = dg::SmemLayout<kBN, kSwap, kStages, kCtaGroup, kSwap && kLayout == dg::kDense && kBN <= 128>;
     auto kernel = dg::fp8_gemm_kernel<kBN, kSwap, kStages, kLayout, kCtaGroup, kSwiGLU>;
     static bool attr_done[kMaxDevices] = {};
@@ -219,7 +247,7 @@ dg_status_t launch(const CUtensorMap &ma, const CUtensorMap &mb, const dg::Param
                      "split=%d grid=%dx%d cluster=%d smem=%d\n",
                      kLayout, p.M, p.N, p.K, p.G, kBN, int(kSwap), kStages, kCtaGroup, p.split, grid_x,
                      grid_y, cluster_x, L::kAlloc);
-    cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, ma, mb, p);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, ma, mb, md, p);
     if (e != cudaSuccess) return cuda_fail(e, "cudaLaunchKernelEx");
     return DG_SUCCESS;
 }
@@ -324,6 +352,8 @@ dg_status_t dg_fp8_gemm_nt(const uint8_t *a, const float *sfa, int ld_sfa, const
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     dg::Params p = base_params(sfa, ld_sfa, sfb, d, M, N, K, 1, info);
     CUtensorMap ma, mb;
+    CUtensorMap md;
+    if ((st = make_d_map(&md, d, N, M)) != DG_SUCCESS) return st;
     if (M <= 256) {
         // swap-AB: weights on the 128 TMEM lanes, the few tokens on the MMA's N side
         const int bn = M <= 64 ? 64 : (M <= 128 ? 128 : 256);
@@ -335,16 +365,16 @@ dg_status_t dg_fp8_gemm_nt(const uint8_t *a, const float *sfa, int ld_sfa, const
         if ((st = make_map(&ma, a, K, M, 1, 32)) != DG_SUCCESS) return st;   // 32-token boxes
         const int gx = p.split > 1 ? p.split : (tiles < info->num_sms ? tiles : info->num_sms);
         const int gy = p.split > 1 ? tiles : 1;
-        if (bn == 64) return launch<64, true, 7, dg::kDense>(ma, mb, p, gx, gy, p.split, s);
-        if (bn == 128) return launch<128, true, 4, dg::kDense>(ma, mb, p, gx, gy, p.split, s);
-        return launch<256, true, 4, dg::kDense>(ma, mb, p, gx, gy, p.split, s);
+        if (bn == 64) return launch<64, true, 7, dg::kDense>(ma, mb, md, p, gx, gy, p.split, s);
+        if (bn == 128) return launch<128, true, 4, dg::kDense>(ma, mb, md, p, gx, gy, p.split, s);
+        return launch<256, true, 4, dg::kDense>(ma, mb, md, p, gx, gy, p.split, s);
     }
     if (N <= 128) {
         const int tiles = ((M + 127) / 128) * ((N + 127) / 128);
         const int grid = tiles < info->num_sms ? tiles : info->num_sms;
         if ((st = make_map(&ma, a, K, M, 1, 128)) != DG_SUCCESS) return st;
         if ((st = make_map(&mb, b, K, N, 1, 128)) != DG_SUCCESS) return st;
-        return launch<128, false, 6, dg::kDense>(ma, mb, p, grid, 1, 1, s);
+        return launch<128, false, 6, dg::kDense>(ma, mb, md, p, grid, 1, 1, s);
     }
     // CTA pairs: 256 x bn tiles with tcgen05.mma.cta_group::2 (DG_PAIR_N
     // overrides bn for tuning sweeps)
@@ -365,9 +395,9 @@ dg_status_t dg_fp8_gemm_nt(const uint8_t *a, const float *sfa, int ld_sfa, const
     const int pairs = tiles < pairs_max ? tiles : pairs_max;
     if ((st = make_map(&ma, a, K, M, 1, 128)) != DG_SUCCESS) return st;
     if ((st = make_map(&mb, b, K, N, 1, bn / 2)) != DG_SUCCESS) return st;
-    if (bn == 160) return launch<160, false, 7, dg::kDense, 2>(ma, mb, p, 2 * pairs, 1, 2, s);
-    if (bn == 224) return launch<224, false, 6, dg::kDense, 2>(ma, mb, p, 2 * pairs, 1, 2, s);
-    return launch<256, false, 6, dg::kDense, 2>(ma, mb, p, 2 * pairs, 1, 2, s);
+    if (bn == 160) return launch<160, false, 7, dg::kDense, 2>(ma, mb, md, p, 2 * pairs, 1, 2, s);
+    if (bn == 224) return launch<224, false, 6, dg::kDense, 2>(ma, mb, md, p, 2 * pairs, 1, 2, s);
+    return launch<256, false, 6, dg::kDense, 2>(ma, mb, md, p, 2 * pairs, 1, 2, s);
 }
 
 dg_status_t dg_m_grouped_fp8_gemm_nt_contiguous(const uint8_t *a, const float *sfa, int ld_sfa,
@@ -385,6 +415,8 @@ dg_status_t dg_m_grouped_fp8_gemm_nt_contiguous(const uint8_t *a, const float *s
     dg::Params p = base_params(sfa, ld_sfa, sfb, d, M_total, N, K, G, info);
     p.m_indices = m_indices;
     CUtensorMap ma, mb;
+    CUtensorMap md;
+    if ((st = make_d_map(&md, d, N, M_total)) != DG_SUCCESS) return st;
     // CTA pairs for the contiguous layout measured no faster than 128 x 256
     // single-CTA tiles on the 4-group workload (both are bound by the MMA /
     // promotion hand-off, not by operand traffic); DG_CONTIG_PAIRS=1 selects them.
@@ -406,8 +438,8 @@ dg_status_t dg_m_grouped_fp8_gemm_nt_contiguous(const uint8_t *a, const float *s
             const int pairs = tiles < pairs_max ? static_cast<int>(tiles) : pairs_max;
             if ((st = make_map(&ma, a, K, M_total, 1, 128)) != DG_SUCCESS) return st;
             if ((st = make_map(&mb, b, K, N, G, bn / 2)) != DG_SUCCESS) return st;
-            if (bn == 224) return launch<224, false, 6, dg::kContiguous, 2>(ma, mb, p, 2 * pairs, 1, 2, s);
-            return launch<256, false, 6, dg::kContiguous, 2>(ma, mb, p, 2 * pairs, 1, 2, s);
+            if (bn == 224) return launch<224, false, 6, dg::kContiguous, 2>(ma, mb, md, p, 2 * pairs, 1, 2, s);
+            return launch<256, false, 6, dg::kContiguous, 2>(ma, mb, md, p, 2 * pairs, 1, 2, s);
         }
     }
     const int bn = N <= 128 ? 128 : 256;
@@ -415,8 +447,8 @@ dg_status_t dg_m_grouped_fp8_gemm_nt_contiguous(const uint8_t *a, const float *s
     const int grid = tiles < info->num_sms ? tiles : info->num_sms;
     if ((st = make_map(&ma, a, K, M_total, 1, 128)) != DG_SUCCESS) return st;
     if ((st = make_map(&mb, b, K, N, G, bn)) != DG_SUCCESS) return st;
-    if (bn == 128) return launch<128, false, 6, dg::kContiguous>(ma, mb, p, grid, 1, 1, s);
-    return launch<256, false, 4, dg::kContiguous>(ma, mb, p, grid, 1, 1, s);
+    if (bn == 128) return launch<128, false, 6, dg::kContiguous>(ma, mb, md, p, grid, 1, 1, s);
+    return launch<256, false, 4, dg::kContiguous>(ma, mb, md, p, grid, 1, 1, s);
 }
 
 dg_status_t dg_m_grouped_fp8_gemm_nt_masked(const uint8_t *a, const float *sfa, int ld_sfa,
@@ -434,6 +466,8 @@ dg_status_t dg_m_grouped_fp8_gemm_nt_masked(const uint8_t *a, const float *sfa, 
     dg::Params p = base_params(sfa, ld_sfa, sfb, d, Mmax, N, K, G, info);
     p.masked_m = masked_m;
     CUtensorMap ma, mb;
+    CUtensorMap md;
+    if ((st = make_d_map(&md, d, N, static_cast<long long>(G) * Mmax)) != DG_SUCCESS) return st;
     const int grid = info->num_sms;   // the tile count lives on the device
     static const bool force_swap = [] {
         const char *e = std::getenv("DG_MASKED_SWAP");
@@ -444,8 +478,8 @@ dg_status_t dg_m_grouped_fp8_gemm_nt_masked(const uint8_t *a, const float *sfa, 
         const int bn = Mmax <= 64 ? 64 : 128;
         if ((st = make_map(&mb, b, K, N, G, 128)) != DG_SUCCESS) return st;
         if ((st = make_map(&ma, a, K, Mmax, G, 32)) != DG_SUCCESS) return st;   // 32-token boxes
-        if (bn == 64) return launch<64, true, 8, dg::kMasked>(ma, mb, p, grid, 1, 1, s);
-        return launch<128, true, 6, dg::kMasked>(ma, mb, p, grid, 1, 1, s);
+        if (bn == 64) return launch<64, true, 8, dg::kMasked>(ma, mb, md, p, grid, 1, 1, s);
+        return launch<128, true, 6, dg::kMasked>(ma, mb, md, p, grid, 1, 1, s);
     }
     // Normal mode: 128 token rows on the TMEM lanes, so each promotion thread's
     // token scale is one register and the weight scale is uniform per 128
@@ -464,8 +498,8 @@ dg_status_t dg_m_grouped_fp8_gemm_nt_masked(const uint8_t *a, const float *sfa, 
     if (forced_bn == 128 || forced_bn == 256) bn = forced_bn;
     if ((st = make_map(&ma, a, K, Mmax, G, 128)) != DG_SUCCESS) return st;
     if ((st = make_map(&mb, b, K, N, G, bn)) != DG_SUCCESS) return st;
-    if (bn == 128) return launch<128, false, 6, dg::kMasked>(ma, mb, p, grid, 1, 1, s);
-    return launch<256, false, 4, dg::kMasked>(ma, mb, p, grid, 1, 1, s);
+    if (bn == 128) return launch<128, false, 6, dg::kMasked>(ma, mb, md, p, grid, 1, 1, s);
+    return launch<256, false, 4, dg::kMasked>(ma, mb, md, p, grid, 1, 1, s);
 }
 
 dg_status_t dg_k_grouped_fp8_gemm_nt_contiguous(const uint8_t *a, const float *sfa, int ld_sfa,
@@ -483,6 +517,8 @@ dg_status_t dg_k_grouped_fp8_gemm_nt_contiguous(const uint8_t *a, const float *s
     dg::Params p = base_params(sfa, ld_sfa, sfb, d, M, N, K, G, info);
     p.ks = ks;
     CUtensorMap ma, mb;
+    CUtensorMap md;
+    if ((st = make_d_map(&md, d, N, static_cast<long long>(G) * M)) != DG_SUCCESS) return st;
     if ((st = make_map(&ma, a, K, M, 1, 128)) != DG_SUCCESS) return st;
     // The tile grid does not depend on the group sizes (they only set each
     // tile's K range, read on the device): G x token blocks x weight blocks.
@@ -491,8 +527,8 @@ dg_status_t dg_k_grouped_fp8_gemm_nt_contiguous(const uint8_t *a, const float *s
         const long long tiles = static_cast<long long>(G) * ((M + 127) / 128) * ((N + bn - 1) / bn);
         const int grid = tiles < info->num_sms ? static_cast<int>(tiles) : info->num_sms;
         if ((st = make_map(&mb, b, K, N, 1, bn)) != DG_SUCCESS) return st;
-        if (bn == 128) return launch<128, false, 6, dg::kKGrouped>(ma, mb, p, grid, 1, 1, s);
-        return launch<256, false, 4, dg::kKGrouped>(ma, mb, p, grid, 1, 1, s);
+        if (bn == 128) return launch<128, false, 6, dg::kKGrouped>(ma, mb, md, p, grid, 1, 1, s);
+        return launch<256, false, 4, dg::kKGrouped>(ma, mb, md, p, grid, 1, 1, s);
     }
     // CTA pairs: 256 x bn tiles (tcgen05.mma.cta_group::2), as for large dense GEMMs
     const long long row_pairs = static_cast<long long>(G) * ((M + 255) / 256);
@@ -505,8 +541,8 @@ dg_status_t dg_k_grouped_fp8_gemm_nt_contiguous(const uint8_t *a, const float *s
     const long long tiles = row_pairs * ((N + bn - 1) / bn);
     const int pairs = tiles < pairs_max ? static_cast<int>(tiles) : pairs_max;
     if ((st = make_map(&mb, b, K, N, 1, bn / 2)) != DG_SUCCESS) return st;
-    if (bn == 224) return launch<224, false, 6, dg::kKGrouped, 2>(ma, mb, p, 2 * pairs, 1, 2, s);
-    return launch<256, false, 6, dg::kKGrouped, 2>(ma, mb, p, 2 * pairs, 1, 2, s);
+    if (bn == 224) return launch<224, false, 6, dg::kKGrouped, 2>(ma, mb, md, p, 2 * pairs, 1, 2, s);
+    return launch<256, false, 6, dg::kKGrouped, 2>(ma, mb, md, p, 2 * pairs, 1, 2, s);
 }
 
 dg_status_t dg_m_grouped_fp8_gemm_swiglu_quant_contiguous(
@@ -529,11 +565,13 @@ dg_status_t dg_m_grouped_fp8_gemm_swiglu_quant_contiguous(
     p.s_out = s_out;
     p.ld_s_out = ld_s_out;
     CUtensorMap ma, mb;
+    CUtensorMap md;
+    if ((st = make_d_map(&md, nullptr, N, 0)) != DG_SUCCESS) return st;
     if ((st = make_map(&ma, a, K, M_total, 1, 128)) != DG_SUCCESS) return st;
     if ((st = make_map(&mb, b, K, N, G, 256)) != DG_SUCCESS) return st;
     const int tiles = (M_total / 128) * (N / 256);
     const int grid = tiles < info->num_sms ? tiles : info->num_sms;
-    return launch<256, false, 4, dg::kContiguous, 1, true>(ma, mb, p, grid, 1, 1, static_cast<cudaStream_t>(stream));
+    return launch<256, false, 4, dg::kContiguous, 1, true>(ma, mb, md, p, grid, 1, 1, static_cast<cudaStream_t>(stream));
 }
 
 dg_status_t dg_m_grouped_fp8_ffn_contiguous(const uint8_t *a, const float *sfa, int ld_sfa,

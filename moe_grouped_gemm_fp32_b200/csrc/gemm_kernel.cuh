@@ -358,7 +358,12 @@ struct SmemLayout {
     static constexpr int kRecvRows = 136;
     static constexpr int kRecvOffset = (kPrefixOffset + kPrefixBytes + 127) / 128 * 128;
     static constexpr int kRecvBytes = kSplitK ? kRecvRows * kRecvStride * 4 : 0;
-    static constexpr int kUsed = kRecvOffset + kRecvBytes;
+    // normal mode: per promotion warp a 32-row x 32-column BF16 staging box
+    // (64-byte rows, 64B swizzle) for the TMA-store epilogue
+    static constexpr int kOutBoxBytes = 32 * 64;
+    static constexpr int kOutOffset = (kRecvOffset + kRecvBytes + 1023) / 1024 * 1024;
+    static constexpr int kOutBytes = kSwap ? 0 : 8 * kOutBoxBytes;
+    static constexpr int kUsed = kOutOffset + kOutBytes;
     static constexpr int kAlloc = (kUsed + 1024 > kMinSmem) ? kUsed + 1024 : kMinSmem;
     static constexpr int kTmemCols = kAccBufs * kBN <= 32    ? 32
                                      : kAccBufs * kBN <= 64  ? 64
@@ -370,13 +375,14 @@ struct SmemLayout {
     static_assert(kBarOffset % 8 == 0, "mbarriers are 8-byte objects");
     static_assert(kPrefixOffset % 16 == 0, "prefix table alignment");
     static_assert(kRecvOffset % 16 == 0, "split-K pushes and reads are 16-byte vectors");
+    static_assert(kOutOffset % 1024 == 0, "swizzled TMA-store boxes need aligned shared memory");
     static_assert(kAlloc <= 227 * 1024, "shared memory budget");
 };
 
 template <int kBN, bool kSwap, int kStages, int kLayout, int kCtaGroup, bool kSwiGLU = false>
 __global__ void __launch_bounds__(num_threads(kSwap), 1)
 fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
-                const Params p) {
+                const __grid_constant__ CUtensorMap tm_d, const Params p) {
     // SwiGLU epilogue: a 256-column tile is one 128-row gate block of the
     // weights followed by the matching 128-row up block; each promotion
     // warpgroup owns 64 gate columns and the 64 up columns they pair with
@@ -977,6 +983,12 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
             if (clustered) break;   // one tile; reduced below
             // ------------------------------------------------ epilogue (direct)
             const size_t row_base = (kLayout == kMasked || kLayout == kKGrouped) ? static_cast<size_t>(tl.g) * p.M : 0;
+            // the TMA store may write every row of this CTA's 128-row block:
+            // dense (rows past M are outside the D map), contiguous (padding rows
+            // are don't-care), masked and K-grouped only when the block is full
+            const bool tma_epilogue = !kSwap && ((tl.store >> pair_rank) & 1) != 0 &&
+                                      (kLayout == kDense || kLayout == kContiguous ||
+                                       tl.tok0 + my_row0 + kTileX <= tl.tok_end);
             if constexpr (kSwiGLU) {
                 // act = silu(gate) * up for this thread's 64 columns of the tile's
                 // 128-column activation block; the block's amax is combined with
@@ -1020,6 +1032,62 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
                     }
                     if (half == 0) p.s_out[static_cast<size_t>(ablk) * p.ld_s_out + row_base + my_tok] = sc;
                 }
+            } else if (!kSwap && tma_epilogue) {
+                // TMA-store epilogue: each warp converts its 32 rows x 32 columns
+                // to BF16 in a 64B-swizzled staging box and one lane stores the box
+                // with cp.async.bulk.tensor (rows past M and columns past N fall
+                // outside the D map and are not written)
+                uint8_t *box = smem + L::kOutOffset + (warp - kPromoWarp0) * L::kOutBoxBytes;
+                const uint32_t box_s = ptx::smem_u32(box);
+                const int wrow = tl.tok0 + my_row0 + quarter * 32;     // this warp's first tile row
+                const bool rows_in = kLayout == kMasked || kLayout == kKGrouped || wrow < p.M;
+                const int drow0 = static_cast<int>(row_base) + wrow;    // its row in the D map
+                const int sw = (lane >> 1) & 3;                         // 64B swizzle of this lane's row
+                constexpr int kFull = kHalf / 32;
+#pragma unroll
+                for (int c = 0; c < kFull; ++c) {
+                    uint32_t w[16];
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        __nv_bfloat162 h2 = __floats2bfloat162_rn(acc[c * 32 + 2 * j], acc[c * 32 + 2 * j + 1]);
+                        w[j] = *reinterpret_cast<uint32_t *>(&h2);
+                    }
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        *reinterpret_cast<uint4 *>(box + lane * 64 + ((q ^ sw) * 16)) =
+                            make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+                    ptx::fence_proxy_async_smem();
+                    __syncwarp();
+                    const int col0 = tl.n0 + half * kHalf + c * 32;
+                    if (lane == 0 && rows_in && col0 < p.N) {
+                        ptx::tma_store_2d(&tm_d, box_s, col0, drow0);
+                        ptx::bulk_commit();
+                        ptx::bulk_wait_read0();          // the box may be rewritten
+                    }
+                    __syncwarp();
+                }
+                if constexpr (kHalf % 32 != 0) {
+                    // the 16-column remainder of a 224-wide pair tile: direct stores
+                    if (tok_ok) {
+                        __nv_bfloat16 *drow = p.d + (row_base + my_tok) * static_cast<size_t>(p.N);
+#pragma unroll
+                        for (int j = kFull * 32; j < kHalf; j += 8) {
+                            const int col = tl.n0 + half * kHalf + j;
+                            if (col < p.N) {
+                                uint4 pk;
+                                __nv_bfloat162 h0 = __floats2bfloat162_rn(acc[j + 0], acc[j + 1]);
+                                __nv_bfloat162 h1 = __floats2bfloat162_rn(acc[j + 2], acc[j + 3]);
+                                __nv_bfloat162 h2 = __floats2bfloat162_rn(acc[j + 4], acc[j + 5]);
+                                __nv_bfloat162 h3 = __floats2bfloat162_rn(acc[j + 6], acc[j + 7]);
+                                pk.x = *reinterpret_cast<uint32_t *>(&h0);
+                                pk.y = *reinterpret_cast<uint32_t *>(&h1);
+                                pk.z = *reinterpret_cast<uint32_t *>(&h2);
+                                pk.w = *reinterpret_cast<uint32_t *>(&h3);
+                                *reinterpret_cast<uint4 *>(drow + col) = pk;
+                            }
+                        }
+                    }
+                }
             } else if (!kSwap) {
                 if (tok_ok) {
                     __nv_bfloat16 *drow = p.d + (row_base + my_tok) * static_cast<size_t>(p.N);
@@ -1058,6 +1126,8 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
                 }
             }
         }
+        // every TMA store of this warp has completed before the CTA can exit
+        if (!kSwap && lane == 0) ptx::bulk_wait0();
     }
 
     // ============================================================ split-K reduction
