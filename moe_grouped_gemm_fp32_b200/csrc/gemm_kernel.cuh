@@ -439,30 +439,35 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
     auto leader_addr = [&](uint32_t local) { return kPair ? ptx::map_cluster(local, 0) : local; };
 
     // ------------------------------------------------------------ set-up
-    if (threadIdx.x == 0) {
-        ptx::prefetch_tmap(&tm_a);
-        ptx::prefetch_tmap(&tm_b);
-        for (int s = 0; s < kStages; ++s) {
+    // warp 0 initialises the barriers, one lane per barrier (dozens of them in
+    // swap mode: initialised one after another they delay the first load)
+    if (warp == 0) {
+        if (lane == 0) {
+            ptx::prefetch_tmap(&tm_a);
+            ptx::prefetch_tmap(&tm_b);
+            *abort_flag = 0;
+        }
+        for (int s = lane; s < kStages; s += 32) {
             ptx::mbar_init(full_bar(s), 1);
             // MMA commit (+ 8 promotion warps that read the stage's scales, normal mode)
             ptx::mbar_init(empty_bar(s), kSwap ? 1 : 1 + 8);
         }
         if constexpr (kSwap) {
-            for (int i = 0; i < kSlots; ++i) {
+            for (int i = lane; i < kSlots; i += 32) {
                 ptx::mbar_init(sfull_bar(i), 1);
                 ptx::mbar_init(sready_bar(i), 32);
                 ptx::mbar_init(sempty_bar(i), 8);
             }
         }
-        for (int b = 0; b < kAccBufs; ++b) {
-            ptx::mbar_init(tfull_bar(b), 1);
-            ptx::mbar_init(tempty_bar(b), 8 * kCtaGroup);   // every promotion warp of the pair
+        if (lane < kAccBufs) {
+            ptx::mbar_init(tfull_bar(lane), 1);
+            ptx::mbar_init(tempty_bar(lane), 8 * kCtaGroup);   // every promotion warp of the pair
         }
-        ptx::mbar_init(mma_done_bar, 1);
-        ptx::mbar_init(xchg_bar(0), 256);     // both promotion warpgroups
-        ptx::mbar_init(xchg_bar(1), 256);
-        *abort_flag = 0;
+        if (lane == 31) ptx::mbar_init(mma_done_bar, 1);
+        if (lane == 30) ptx::mbar_init(xchg_bar(0), 256);     // both promotion warpgroups
+        if (lane == 29) ptx::mbar_init(xchg_bar(1), 256);
         ptx::fence_mbar_init();
+        __syncwarp();
     }
     if (kLayout == kMasked && warp == kPromoWarp0) {
         // exclusive prefix of tiles per group: ceil(masked_m[g] / kTokRows) * weight blocks
@@ -557,7 +562,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
     }
     ptx::tc_fence_before();
     if constexpr (kEarly) {
-        // warp 0 (the producer; thread 0 initialised the barriers) arrives and
+        // warp 0 (the producer; it initialised the barriers) arrives and
         // goes on; the other warps wait until the barriers and TMEM are ready
         if (warp == 0) ptx::named_bar_arrive(1, num_threads(kSwap));
         else ptx::named_bar_sync(1, num_threads(kSwap));
@@ -590,7 +595,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
     if constexpr (!kSwap) ptx::regs_dec<kRegsIssue>();
     if (warp == 0) {
         // ======================================================== producer
-        // (one elected thread; the warp-wide sync orders it after thread 0's
+        // (one elected thread; the warp-wide sync orders it after the warp's
         // barrier initialisation when the producer starts before the set-up barrier)
         __syncwarp();
         if (ptx::elect_one()) {
