@@ -417,13 +417,17 @@ dg_status_t dg_m_grouped_fp8_gemm_nt_contiguous(const uint8_t *a, const float *s
     CUtensorMap ma, mb;
     CUtensorMap md;
     if ((st = make_d_map(&md, d, N, M_total)) != DG_SUCCESS) return st;
-    // CTA pairs for the contiguous layout measured no faster than 128 x 256
-    // single-CTA tiles on the 4-group workload (both are bound by the MMA /
-    // promotion hand-off, not by operand traffic); DG_CONTIG_PAIRS=1 selects them.
-    static const bool contig_pairs = [] {
+    // CTA pairs (256-row tiles) by default for N > 128 and K >= 4096: with the
+    // TMA-store epilogue they measured 997 us against 1018 us for 128 x 256
+    // single-CTA tiles on 4 groups x 32768 tokens x N 4096 x K 7168, but were
+    // slower with short K (the FFN's down projection, K 2048: fewer K-blocks
+    // per tile to amortise the pair's tile switch).  DG_CONTIG_PAIRS=0 / =1
+    // forces single-CTA tiles / pairs.
+    static const int contig_pairs_env = [] {
         const char *e = std::getenv("DG_CONTIG_PAIRS");
-        return e && e[0] == '1';
+        return e ? (e[0] == '1' ? 1 : 0) : -1;
     }();
+    const bool contig_pairs = contig_pairs_env >= 0 ? contig_pairs_env == 1 : K >= 4096;
     if (contig_pairs && N > 128 && G < dg::kMaxGroups) {
         // CTA pairs with 256-row tiles; pairs straddling a group boundary run
         // a second pass (the tile count grows by at most (G-1) x N-tiles)

@@ -112,8 +112,19 @@ def test_contiguous(counts, N, K):
 
 @pytest.mark.parametrize("counts,N,K", [([130, 200, 5, 300, 129], 448, 384), ([128, 256], 2112, 512)])
 def test_contiguous_cta_pairs(counts, N, K):
-    """The CTA-pair contiguous path (opt-in) in a child process: second passes
-    for pair tiles whose two 128-row blocks belong to different groups."""
+    """The CTA-pair contiguous path (the default for N > 128 and K >= 4096),
+    forced on at small K in a child process: second passes for pair tiles
+    whose two 128-row blocks belong to different groups."""
+    _run_contiguous_child(counts, N, K, pairs=True)
+
+
+@pytest.mark.parametrize("counts,N,K", [([130, 200, 5, 300, 129], 384, 4096), ([1] * 7, 256, 4096)])
+def test_contiguous_single_cta_tiles(counts, N, K):
+    """The single-CTA contiguous path forced at long K in a child process."""
+    _run_contiguous_child(counts, N, K, pairs=False)
+
+
+def _run_contiguous_child(counts, N, K, pairs):
     import os, subprocess, sys
     code = ("import sys; sys.path[:0] = [%r, %r]\n"
             "import workloads as W, oracle\n"
@@ -122,10 +133,15 @@ def test_contiguous_cta_pairs(counts, N, K):
             "dp = DeviceProblem(p); dp.fill_sentinel(); d = to_f64(dp.run())\n"
             "compare(d, oracle.solve(p), valid_mask(p)); print('OK')\n"
             % (os.path.dirname(os.path.dirname(__file__)), os.path.dirname(__file__), counts, N, K))
-    env = dict(os.environ, DG_CONTIG_PAIRS="1", DG_VERBOSE="1")
+    env = dict(os.environ, DG_CONTIG_PAIRS="1" if pairs else "0", DG_VERBOSE="1")
     r = subprocess.run([sys.executable, "-c", code], env=env, capture_output=True, text=True, timeout=300)
     assert r.returncode == 0 and "OK" in r.stdout, r.stdout + r.stderr
-    assert "ctas/mma=2" in r.stderr
+    assert ("ctas/mma=2" if pairs else "ctas/mma=1") in r.stderr
+
+
+def test_contiguous_long_k_default_pairs():
+    """K >= 4096 takes CTA pairs by default (group boundaries inside pair tiles)."""
+    _run_full(W.make_contiguous([130, 200, 5, 300, 129], 448, 4096, seed=91))
 
 
 def test_contiguous_multinomial_small():
