@@ -77,7 +77,8 @@ constexpr int kTokBox = 32;          // swap mode: token rows per TMA box
 enum StatusCode : unsigned { kStatusInvalid = 1u, kStatusTimeout = 6u };
 enum Site : unsigned {
     kSiteProducerEmpty = 1, kSiteMmaTmemEmpty = 2, kSiteMmaFull = 3, kSitePromoFull = 4,
-    kSiteTeardownLoads = 5, kSiteTeardownMma = 6, kSiteBadGroup = 7, kSiteBadMask = 8, kSiteBadKs = 10
+    kSiteTeardownLoads = 5, kSiteTeardownMma = 6, kSiteBadGroup = 7, kSiteBadMask = 8, kSiteBadKs = 10,
+    kSiteSplitKRecv = 11
 };
 
 struct Params {
@@ -347,8 +348,9 @@ struct SmemLayout {
     // Each K-block's partial lives from its MMA until the promotion warps have
     // read it; more buffers let the MMAs run further ahead of the promotion.
     static constexpr int kAccBufs = 512 / kBN >= 4 ? 4 : (512 / kBN >= 3 ? 3 : 2);
-    // + 2: the SwiGLU epilogue's amax-exchange barriers (one per tile parity)
-    static constexpr int kNumBars = 2 * kStages + 2 * kAccBufs + 1 + (kSwap ? 3 * kSlots : 0) + 2;
+    // + 3: the split-K receive barrier and the SwiGLU epilogue's amax-exchange
+    // barriers (one per tile parity)
+    static constexpr int kNumBars = 2 * kStages + 2 * kAccBufs + 1 + (kSwap ? 3 * kSlots : 0) + 3;
     static constexpr int kMiscOffset = kBarOffset + kNumBars * 8;     // tmem addr, abort flag
     static constexpr int kPrefixOffset = (kMiscOffset + 16 + 15) / 16 * 16;
     static constexpr int kPrefixBytes = (kMaxGroups + 1) * 4;
@@ -424,6 +426,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
     auto sready_bar = [&](int i) { return bar_base + 8u * (2 * kStages + 2 * kAccBufs + 1 + kSlots + i); };
     auto sempty_bar = [&](int i) { return bar_base + 8u * (2 * kStages + 2 * kAccBufs + 1 + 2 * kSlots + i); };
     auto xchg_bar = [&](int i) { return bar_base + 8u * (L::kNumBars - 2 + i); };
+    const uint32_t recv_bar = bar_base + 8u * (L::kNumBars - 3);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kMiscOffset);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kMiscOffset + 4);
     const uint32_t slot_base = s_base + L::kSlotOffset;
@@ -466,6 +469,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
         if (lane == 31) ptx::mbar_init(mma_done_bar, 1);
         if (lane == 30) ptx::mbar_init(xchg_bar(0), 256);     // both promotion warpgroups
         if (lane == 29) ptx::mbar_init(xchg_bar(1), 256);
+        if (lane == 28) ptx::mbar_init(recv_bar, 1);     // split-K: the owner's expect-tx arrival
         ptx::fence_mbar_init();
         __syncwarp();
     }
@@ -579,6 +583,11 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
     const int t_first = clustered ? static_cast<int>(blockIdx.y) : static_cast<int>(blockIdx.x) / kCtaGroup;
     const int t_step = clustered ? num_tiles : static_cast<int>(gridDim.x) / kCtaGroup;
     int kb_begin = 0, kb_end = p.num_kb;
+    // split-K: every CTA's barriers exist before any other CTA of the cluster
+    // signals them (their initialisation was fenced with release at cluster
+    // scope, so a relaxed arrival suffices); the wait comes just before the
+    // exchange, long after, so nobody stalls here
+    if (clustered) ptx::cluster_arrive_relaxed();
     if (clustered) {
         const int r = static_cast<int>(ptx::cluster_rank());
         kb_begin = (p.num_kb * r) / p.split;
@@ -741,9 +750,9 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
         __syncwarp();
     }
 
-    if (clustered) {   // the split-K exchange barrier of the promotion warps
+    if (clustered) {   // completes the set-up arrival (matches the promotion warps)
         __syncwarp();
-        ptx::cluster_sync_all();
+        ptx::cluster_wait_acquire();
     }
     // ------------------------------------------------------------ teardown (issue warps)
     if (warp == 1 && ptx::elect_one()) {
@@ -759,6 +768,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
         }
     }
     __syncwarp();
+    if (clustered) ptx::cluster_sync_all();   // split-K: the exchange's final barrier
     ptx::tc_fence_before();
     __syncthreads();
     if constexpr (kPair) ptx::cluster_sync_all();   // no CTA leaves while its peer may touch its smem
@@ -790,8 +800,9 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
             }
         }
     }
-    if (clustered) {   // the split-K exchange barrier of the promotion warps
+    if (clustered) {   // completes the set-up arrival, then the exchange's final barrier
         __syncwarp();
+        ptx::cluster_wait_acquire();
         ptx::cluster_sync_all();
     }
     ptx::tc_fence_before();
@@ -1137,51 +1148,78 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
 
     // ============================================================ split-K reduction
     if (clustered) {
-        // (1) push this thread's row to its owner's receive buffer, slot
-        // [source rank][owned row][column].  The buffer is private to the split-K
-        // exchange, so no CTA waits for the others before writing.
+        // Rows are owned in blocks of rows_per by the cluster's ranks.  (1) each
+        // CTA stages its FP32 partial tile row-major ([weight row][token], rows
+        // padded to kRecvStride floats) in the idle operand stages; (2) one thread
+        // ships each owner's rows with one bulk copy into the owner's receive
+        // buffer, slot [source rank][owned row][token], completing on the owner's
+        // receive barrier; (3) the owner waits for the other ranks' bytes
+        // (bounded) and sums in rank order.  No per-thread remote stores, and no
+        // cluster-wide barrier before the reduction.
         const int split = p.split;
         const int rows_per = (kTileX + split - 1) / split;     // the last owner may get fewer
         const uint32_t my_rank = ptx::cluster_rank();
         const uint32_t recv_base = s_base + L::kRecvOffset;
-        if (have_tile && !*abort_flag) {
-            const int owner = lrow / rows_per;
-            const uint32_t local = recv_base + static_cast<uint32_t>(
-                ((my_rank * rows_per + (lrow - owner * rows_per)) * L::kRecvStride) * 4);
-            const uint32_t remote = ptx::map_cluster(local, static_cast<uint32_t>(owner));
+        const uint32_t row_bytes = L::kRecvStride * 4;
+        float *stg = reinterpret_cast<float *>(smem);          // operand stages: all loads consumed
+        const bool sending = have_tile && !*abort_flag;
+        if (sending) {
+            float *row = stg + lrow * L::kRecvStride;
 #pragma unroll
             for (int c = 0; c < kChunks; ++c) {
                 if (c < last_nvalid) {
 #pragma unroll
                     for (int i = 0; i < kChunk; i += 4)
-                        ptx::st_cluster_v4(remote + (col_of(c) + i) * 4, acc[c * kChunk + i],
-                                           acc[c * kChunk + i + 1], acc[c * kChunk + i + 2],
-                                           acc[c * kChunk + i + 3]);
+                        *reinterpret_cast<float4 *>(row + col_of(c) + i) =
+                            make_float4(acc[c * kChunk + i], acc[c * kChunk + i + 1], acc[c * kChunk + i + 2],
+                                        acc[c * kChunk + i + 3]);
                 }
             }
         }
-        // (2) every push of the cluster has landed
+        ptx::fence_proxy_async_smem();            // the bulk copies read the staging
+        ptx::named_bar_sync(2, 256);              // every promotion thread has staged
         __syncwarp();
-        ptx::cluster_sync_all();
+        ptx::cluster_wait_acquire();              // every CTA's receive barrier exists
+        const int my_rows = max(0, min(rows_per, kTileX - static_cast<int>(my_rank) * rows_per));
+        if (warp == kPromoWarp0 && lane == 0) {
+            if (have_tile && my_rows > 0)
+                ptx::mbar_arrive_expect_tx(recv_bar, static_cast<uint32_t>((split - 1) * my_rows) * row_bytes);
+            if (sending) {
+                for (int o = 0; o < split; ++o) {
+                    const int rows_o = min(rows_per, kTileX - o * rows_per);
+                    if (o == static_cast<int>(my_rank) || rows_o <= 0) continue;
+                    const uint32_t src = s_base + static_cast<uint32_t>(o * rows_per) * row_bytes;
+                    const uint32_t dst = ptx::map_cluster(
+                        recv_base + static_cast<uint32_t>(my_rank * rows_per) * row_bytes, static_cast<uint32_t>(o));
+                    ptx::bulk_copy_to_cluster(dst, src, static_cast<uint32_t>(rows_o) * row_bytes,
+                                              ptx::map_cluster(recv_bar, static_cast<uint32_t>(o)));
+                }
+            }
+        }
+        bool got = true;
+        if (have_tile && my_rows > 0) got = wait(recv_bar, 0u, kSiteSplitKRecv);
         // (3) each CTA sums its rows over the source ranks in rank order and stores.
         // Thread -> (row rr, 4 columns j4): consecutive threads take consecutive rows,
         // so a quarter-warp's 16-byte reads hit distinct banks (padded row stride)
         // and a warp's BF16 stores of one column are contiguous in D.
-        if (have_tile) {
+        if (have_tile && got) {
             const float4 *recv = reinterpret_cast<const float4 *>(smem + L::kRecvOffset);
+            const float4 *own = reinterpret_cast<const float4 *>(stg);
             const Tile &tl = last_tile;
             const size_t row_base = (kLayout == kMasked || kLayout == kKGrouped) ? static_cast<size_t>(tl.g) * p.M : 0;
             const int tid = (warp - kPromoWarp0) * 32 + lane;        // 0..255
-            const int my_rows = min(rows_per, kTileX - static_cast<int>(my_rank) * rows_per);
             const int groups = (tl.ntok + 3) / 4;
-            const int elems = my_rows > 0 ? my_rows * groups : 0;
-            const int n = tl.n0 + static_cast<int>(my_rank) * rows_per;
+            const int elems = my_rows * groups;
+            const int row0 = static_cast<int>(my_rank) * rows_per;
+            const int n = tl.n0 + row0;
             for (int e = tid; e < elems; e += 256) {
                 const int rr = e % my_rows;
                 const int j4 = e / my_rows;
                 float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
                 for (int src = 0; src < split; ++src) {
-                    const float4 v = recv[((src * rows_per + rr) * L::kRecvStride) / 4 + j4];
+                    const float4 v = src == static_cast<int>(my_rank)
+                                         ? own[((row0 + rr) * L::kRecvStride) / 4 + j4]
+                                         : recv[((src * rows_per + rr) * L::kRecvStride) / 4 + j4];
                     sum.x += v.x; sum.y += v.y; sum.z += v.z; sum.w += v.w;
                 }
                 const float vals[4] = {sum.x, sum.y, sum.z, sum.w};
@@ -1195,6 +1233,10 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
                 }
             }
         }
+        // no CTA leaves while a peer's bulk copy may still read its staging or
+        // write its receive buffer
+        __syncwarp();
+        ptx::cluster_sync_all();
     }
 
     // ------------------------------------------------------------ teardown (promotion warps)
