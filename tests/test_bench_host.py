@@ -83,3 +83,39 @@ def test_max_over_ranks_gloo_world_2():
         assert p.exitcode == 0
     res = dict(q.get(timeout=10) for _ in range(2))
     assert res[0] == res[1] == [2.0, 5.0]
+
+
+def test_every_workload_has_a_unit_a_kernel_and_a_config():
+    """Every bench workload resolves to a unit, a profiled kernel name with
+    hashed sources, and a JSON-serialisable shape config; other ranks draw
+    other values of the same shapes."""
+    names = (list(W.WORKLOADS) + list(W.QUANT_WORKLOADS) + list(W.BF16_WORKLOADS) + list(W.FFN_WORKLOADS))
+    small = {"quant_tiny", "bf16_dense_decode_m64", "dense_tiny", "dense_decode_m64"}
+    for w in names:
+        assert w in bench.UNIT, w
+        k = bench.kernel_name(w)
+        assert k in bench.KERNEL_SOURCES and len(bench.kernel_source_hash(k)) == 16
+        if w not in small:
+            continue
+        p0, p1 = bench.rank_problem(w, 0), bench.rank_problem(w, 1)
+        cfg = bench.shape_config(p0)
+        json.dumps(cfg)
+        assert cfg == bench.shape_config(p1)
+        assert p0.bytes() > 0
+        a0 = p0.x if hasattr(p0, "x") else p0.a
+        a1 = p1.x if hasattr(p1, "x") else p1.a
+        assert not np.array_equal(a0, a1)
+
+
+@pytest.mark.parametrize("workload", ["quant_tiny", "bf16_dense_decode_m64"])
+def test_reference_arm_for_the_next_rows(workload):
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--workload", workload, "--steps", "1", "--warmup", "3"],
+                       cwd=ROOT, capture_output=True, text=True, timeout=900)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["config"]["workload"] == workload
+    assert d["value"] > 0 and d["unit"] == bench.UNIT[workload]
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["e2e"]["h2d_bytes_per_step"] == 0
