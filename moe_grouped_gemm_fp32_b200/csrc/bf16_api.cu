@@ -7,6 +7,7 @@
 #include <cuda_runtime.h>
 
 #include <cstdio>
+#include <cstdlib>
 
 #include "dg.h"
 #include "api_common.h"
@@ -41,11 +42,11 @@ dg::Params bf16_params(void *d, int rows, int N, int K, int G, const DeviceInfo 
     return p;
 }
 
-template <int kBN, int kStages, int kLayout>
+template <int kBN, int kStages, int kLayout, bool kSplitK = false>
 dg_status_t launch_bf16(const CUtensorMap &ma, const CUtensorMap &mb, const dg::Params &p, int grid,
-                        cudaStream_t stream) {
-    using L = dg::Bf16Smem<kBN, kStages>;
-    auto kernel = dg::bf16_gemm_kernel<kBN, kStages, kLayout>;
+                        cudaStream_t stream, int grid_y = 1, int cluster_x = 1) {
+    using L = dg::Bf16Smem<kBN, kStages, kSplitK>;
+    auto kernel = dg::bf16_gemm_kernel<kBN, kStages, kLayout, kSplitK>;
     static bool configured[kMaxDevices] = {};
     int dev = 0;
     cudaGetDevice(&dev);
@@ -55,10 +56,24 @@ dg_status_t launch_bf16(const CUtensorMap &ma, const CUtensorMap &mb, const dg::
         configured[dev] = true;
     }
     if (verbose())
-        std::fprintf(stderr, "[dg] bf16_gemm layout=%d bn=%d stages=%d grid=%d smem=%d\n", kLayout, kBN,
-                     kStages, grid, L::kAlloc);
-    kernel<<<grid, dg::kBf16Threads, L::kAlloc, stream>>>(ma, mb, p);
-    cudaError_t e = cudaGetLastError();
+        std::fprintf(stderr, "[dg] bf16_gemm layout=%d bn=%d stages=%d grid=%dx%d cluster=%d split=%d smem=%d\n",
+                     kLayout, kBN, kStages, grid, grid_y, cluster_x, p.split, L::kAlloc);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid, grid_y, 1);
+    cfg.blockDim = dim3(dg::kBf16Threads, 1, 1);
+    cfg.dynamicSmemBytes = L::kAlloc;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    cfg.attrs = attr;
+    cfg.numAttrs = 0;
+    if (cluster_x > 1) {
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = cluster_x;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.numAttrs = 1;
+    }
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, ma, mb, p);
     return e == cudaSuccess ? DG_SUCCESS : cuda_fail(e, "bf16_gemm_kernel launch");
 }
 
@@ -73,6 +88,40 @@ int pick_bn(long long token_blocks, int N, int num_sms) {
         return (static_cast<double>(N) / (nt * bn)) * (static_cast<double>(tiles) / (waves * num_sms));
     };
     return eff(224) > eff(256) + 1e-9 ? 224 : 256;
+}
+
+// Resident clusters of `split` CTAs of the split-K kernel (0 if the query fails).
+template <int kBN, int kStages>
+int bf16_max_clusters(int split) {
+    using L = dg::Bf16Smem<kBN, kStages, true>;
+    auto kernel = dg::bf16_gemm_kernel<kBN, kStages, dg::kDense, true>;
+    static int cache[kMaxDevices][9] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (split < 2 || split > 8) return 0;
+    if (cache[dev][split]) return cache[dev][split];
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc) != cudaSuccess) {
+        cudaGetLastError();
+        return 0;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(split, 1, 1);
+    cfg.blockDim = dim3(dg::kBf16Threads, 1, 1);
+    cfg.dynamicSmemBytes = L::kAlloc;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = split;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, kernel, &cfg) != cudaSuccess) {
+        cudaGetLastError();
+        return 0;
+    }
+    cache[dev][split] = n;
+    return n;
 }
 
 template <int kLayout>
@@ -99,11 +148,36 @@ dg_status_t dg_bf16_gemm_nt(const void *a, const void *b, void *d, int M, int N,
     const DeviceInfo *info = nullptr;
     if ((st = device_info(&info)) != DG_SUCCESS) return st;
     if (M == 0) return DG_SUCCESS;
-    const dg::Params p = bf16_params(d, M, N, K, 1, info);
+    dg::Params p = bf16_params(d, M, N, K, 1, info);
     CUtensorMap ma;
     if ((st = make_kmajor_map(&ma, a, 2, K, M, 1, 128)) != DG_SUCCESS) return st;
-    return dispatch<dg::kDense>(ma, b, N, K, 1, p, (M + 127) / 128, info->num_sms,
-                                static_cast<cudaStream_t>(stream));
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    // one token block and few weight tiles (decode shapes): split K over a
+    // cluster of CTAs per 128-wide tile, the largest split <= 8 whose clusters
+    // are all resident (DG_SPLIT_K overrides)
+    if (M <= 128) {
+        static const int forced = [] {
+            const char *e = std::getenv("DG_SPLIT_K");
+            return e ? std::atoi(e) : 0;
+        }();
+        const int tiles = (N + 127) / 128;
+        int split = 1;
+        if (forced >= 2 && forced <= 8) {
+            split = p.num_kb >= 2 * forced ? forced : 1;
+        } else {
+            for (int c = 8; c >= 2; --c) {
+                if (tiles * c > info->num_sms || p.num_kb < 2 * c) continue;
+                if (bf16_max_clusters<128, 4>(c) >= tiles) { split = c; break; }
+            }
+        }
+        if (split > 1) {
+            CUtensorMap mb;
+            if ((st = make_kmajor_map(&mb, b, 2, K, N, 1, 128)) != DG_SUCCESS) return st;
+            p.split = split;
+            return launch_bf16<128, 4, dg::kDense, true>(ma, mb, p, split, s, tiles, split);
+        }
+    }
+    return dispatch<dg::kDense>(ma, b, N, K, 1, p, (M + 127) / 128, info->num_sms, s);
 }
 
 dg_status_t dg_m_grouped_bf16_gemm_nt_contiguous(const void *a, const void *b, void *d,

@@ -36,30 +36,38 @@ __host__ __device__ constexpr uint32_t bf16_idesc(int m, int n) {
            (static_cast<uint32_t>(m >> 4) << 24);
 }
 
-template <int kBN, int kStages>
+template <int kBN, int kStages, bool kSplitK = false>
 struct Bf16Smem {
     static constexpr int kXBytes = kTileX * 128;        // 128 rows x 64 BF16
     static constexpr int kYBytes = kBN * 128;
     static constexpr int kStageBytes = kXBytes + kYBytes;
     static constexpr int kAccBufs = 2;
     static constexpr int kBarOffset = kStages * kStageBytes;
-    static constexpr int kNumBars = 2 * kStages + 2 * kAccBufs + 1;
+    static constexpr int kNumBars = 2 * kStages + 2 * kAccBufs + 2;   // + split-K receive barrier
     static constexpr int kMiscOffset = kBarOffset + kNumBars * 8;   // tmem addr, abort flag
     static constexpr int kPrefixOffset = (kMiscOffset + 16 + 15) / 16 * 16;
     static constexpr int kPrefixBytes = (kMaxGroups + 1) * 4;
-    static constexpr int kUsed = kPrefixOffset + kPrefixBytes;
+    // split-K: receive buffer [source rank][owned row][column], rows padded by 4
+    // floats; 136 rows cover any split of 128 rows into <= 8 owners
+    static constexpr int kRecvStride = kBN + 4;
+    static constexpr int kRecvOffset = (kPrefixOffset + kPrefixBytes + 127) / 128 * 128;
+    static constexpr int kRecvBytes = kSplitK ? 136 * kRecvStride * 4 : 0;
+    static constexpr int kUsed = kRecvOffset + kRecvBytes;
     static constexpr int kAlloc = (kUsed + 1024 > kMinSmem) ? kUsed + 1024 : kMinSmem;
     static constexpr int kTmemCols = kAccBufs * kBN <= 256 ? 256 : 512;
     static_assert(kAccBufs * kBN <= 512, "TMEM holds 512 columns");
     static_assert(kStageBytes % 1024 == 0, "stage must keep 1024-byte alignment");
     static_assert(kAlloc <= 227 * 1024, "shared memory budget");
+    static_assert(!kSplitK || kTileX * kRecvStride * 4 <= kStages * kStageBytes,
+                  "split-K staging lives in the operand stages");
 };
 
-template <int kBN, int kStages, int kLayout>
+template <int kBN, int kStages, int kLayout, bool kSplitK = false>
 __global__ void __launch_bounds__(kBf16Threads, 1)
 bf16_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                  const Params p) {
-    using L = Bf16Smem<kBN, kStages>;
+    using L = Bf16Smem<kBN, kStages, kSplitK>;
+    static_assert(!kSplitK || kLayout == kDense, "split-K: dense layout");
     using TM = TileMap<kBN, false, kLayout, 1>;
     static_assert(kBN == 128 || kBN == 224 || kBN == 256, "tile N");
     static_assert(kLayout != kKGrouped, "BF16: dense, contiguous and masked layouts");
@@ -76,6 +84,7 @@ bf16_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant
     auto tfull_bar = [&](int b) { return bar_base + 8u * (2 * kStages + b); };
     auto tempty_bar = [&](int b) { return bar_base + 8u * (2 * kStages + kAccBufs + b); };
     const uint32_t mma_done_bar = bar_base + 8u * (2 * kStages + 2 * kAccBufs);
+    const uint32_t recv_bar = bar_base + 8u * (2 * kStages + 2 * kAccBufs + 1);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kMiscOffset);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kMiscOffset + 4);
     int *prefix = reinterpret_cast<int *>(smem + L::kPrefixOffset);
@@ -96,6 +105,7 @@ bf16_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant
             ptx::mbar_init(tempty_bar(b), 4);          // one arrival per epilogue warp
         }
         ptx::mbar_init(mma_done_bar, 1);
+        ptx::mbar_init(recv_bar, 1);               // split-K: the owner's expect-tx arrival
         *abort_flag = 0;
         ptx::fence_mbar_init();
     }
@@ -134,10 +144,22 @@ bf16_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant
     ptx::tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
 
-    const int num_tiles = TM::count(p, prefix);
-    const int t_first = static_cast<int>(blockIdx.x);
-    const int t_step = static_cast<int>(gridDim.x);
-    const int num_kb = p.num_kb;
+    // split-K (dense, few tiles): a cluster of p.split CTAs shares one tile, each
+    // CTA takes a contiguous range of K-blocks; the FP32 partials are summed in
+    // rank order through distributed shared memory (see the epilogue)
+    const bool clustered = kSplitK && p.split > 1;
+    const int num_tiles = clustered ? static_cast<int>(gridDim.y) : TM::count(p, prefix);
+    const int t_first = clustered ? static_cast<int>(blockIdx.y) : static_cast<int>(blockIdx.x);
+    const int t_step = clustered ? num_tiles : static_cast<int>(gridDim.x);
+    int kb_begin = 0, kb_end = p.num_kb;
+    if (clustered) {
+        // every CTA's receive barrier exists before another CTA signals it (its
+        // initialisation was fenced at cluster scope); the wait comes much later
+        ptx::cluster_arrive_relaxed();
+        const int r = static_cast<int>(ptx::cluster_rank());
+        kb_begin = (p.num_kb * r) / p.split;
+        kb_end = (p.num_kb * (r + 1)) / p.split;
+    }
 
     if (warp == 0) {
         // ============================================================ producer
@@ -154,7 +176,7 @@ bf16_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant
                         record_status(p.status, kStatusInvalid, kSiteBadGroup);
                     continue;
                 }
-                for (int kb = 0; kb < num_kb; ++kb) {
+                for (int kb = kb_begin; kb < kb_end; ++kb) {
                     if (!wait(empty_bar(stage), phase ^ 1u, kSiteProducerEmpty)) { ok = false; break; }
                     const uint32_t sx = s_base + stage * L::kStageBytes;
                     ptx::mbar_arrive_expect_tx(full_bar(stage), L::kStageBytes);
@@ -192,7 +214,7 @@ bf16_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant
                 if (!TM::decode(t, p, prefix, tl)) continue;
                 if (!wait(tempty_bar(buf), tphase ^ 1u, kSiteMmaTmemEmpty)) { ok = false; break; }
                 const uint32_t dtm = tmem_base + static_cast<uint32_t>(buf * kBN);
-                for (int kb = 0; kb < num_kb; ++kb) {
+                for (int kb = kb_begin; kb < kb_end; ++kb) {
                     if (!wait(full_bar(stage), phase, kSiteMmaFull)) { ok = false; break; }
                     ptx::tc_fence_after();
                     const uint32_t sx = s_base + stage * L::kStageBytes;
@@ -200,7 +222,7 @@ bf16_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant
                     const uint64_t dy = sw128_desc(sx + L::kXBytes);
 #pragma unroll
                     for (int k = 0; k < kBf16BlockK / 16; ++k)
-                        ptx::mma_f16(dtm, dx + 2u * k, dy + 2u * k, idesc, (kb > 0 || k > 0) ? 1u : 0u);
+                        ptx::mma_f16(dtm, dx + 2u * k, dy + 2u * k, idesc, (kb > kb_begin || k > 0) ? 1u : 0u);
                     ptx::mma_commit(empty_bar(stage));
                     if (++stage == kStages) { stage = 0; phase ^= 1u; }
                 }
@@ -217,6 +239,8 @@ bf16_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant
         const int lrow = quarter * 32 + lane;
         int buf = 0;
         uint32_t tphase = 0;
+        Tile split_tile{};
+        bool have_split_tile = false;
         for (int t = t_first; t < num_tiles; t += t_step) {
             Tile tl;
             if (!TM::decode(t, p, prefix, tl)) continue;
@@ -224,6 +248,23 @@ bf16_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant
             ptx::tc_fence_after();
             const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
                                    static_cast<uint32_t>(buf * kBN);
+            if (clustered) {
+                // stage the FP32 partial tile row-major (rows padded to kRecvStride
+                // floats) in the idle operand stages, then exchange (below)
+                float *row = reinterpret_cast<float *>(smem) + lrow * L::kRecvStride;
+#pragma unroll 1
+                for (int c = 0; c < kBN / 32; ++c) {
+                    float v[32];
+                    ptx::tmem_ld32p(taddr + c * 32, v);
+                    ptx::tmem_wait_ld();
+#pragma unroll
+                    for (int j = 0; j < 32; j += 4)
+                        *reinterpret_cast<float4 *>(row + c * 32 + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+                }
+                split_tile = tl;
+                have_split_tile = true;
+                break;   // one tile per cluster
+            }
             const int my_tok = tl.tok0 + lrow;
             const bool row_ok = my_tok < tl.tok_end;
             const size_t row_base = kLayout == kMasked ? static_cast<size_t>(tl.g) * p.M : 0;
@@ -258,6 +299,86 @@ bf16_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant
             if (lane == 0) ptx::mbar_arrive(tempty_bar(buf));
             if (++buf == kAccBufs) { buf = 0; tphase ^= 1u; }
         }
+        if (clustered) {
+            // Token rows are owned in blocks of rows_per by the cluster's ranks: one
+            // thread ships each owner's rows of this CTA's staged partial with one
+            // bulk copy into the owner's receive buffer, slot [source rank][owned
+            // row][column], completing on the owner's receive barrier; the owner
+            // waits for the other ranks' bytes (bounded), sums in rank order and
+            // stores BF16 rows.
+            const int split = p.split;
+            const Tile &tl = split_tile;
+            const int ntok = have_split_tile ? tl.ntok : 0;
+            const int rows_per = (ntok + split - 1) / split;
+            const uint32_t my_rank = ptx::cluster_rank();
+            const uint32_t row_bytes = L::kRecvStride * 4;
+            const uint32_t recv_base = s_base + L::kRecvOffset;
+            const int my_rows = max(0, min(rows_per, ntok - static_cast<int>(my_rank) * rows_per));
+            const bool sending = have_split_tile && !*abort_flag;
+            ptx::fence_proxy_async_smem();            // the bulk copies read the staging
+            ptx::named_bar_sync(2, 128);              // the four epilogue warps have staged
+            __syncwarp();
+            ptx::cluster_wait_acquire();              // every CTA's receive barrier exists
+            if (warp == kEpiWarp0 && lane == 0) {
+                if (my_rows > 0)
+                    ptx::mbar_arrive_expect_tx(recv_bar, static_cast<uint32_t>((split - 1) * my_rows) * row_bytes);
+                if (sending) {
+                    for (int o = 0; o < split; ++o) {
+                        const int rows_o = min(rows_per, ntok - o * rows_per);
+                        if (o == static_cast<int>(my_rank) || rows_o <= 0) continue;
+                        const uint32_t src = s_base + static_cast<uint32_t>(o * rows_per) * row_bytes;
+                        const uint32_t dst = ptx::map_cluster(
+                            recv_base + static_cast<uint32_t>(my_rank * rows_per) * row_bytes, static_cast<uint32_t>(o));
+                        ptx::bulk_copy_to_cluster(dst, src, static_cast<uint32_t>(rows_o) * row_bytes,
+                                                  ptx::map_cluster(recv_bar, static_cast<uint32_t>(o)));
+                    }
+                }
+            }
+            bool got = true;
+            if (my_rows > 0) got = wait(recv_bar, 0u, kSitePromoFull);
+            if (have_split_tile && got && my_rows > 0) {
+                const float *own = reinterpret_cast<const float *>(smem);
+                const float *recv = reinterpret_cast<const float *>(smem + L::kRecvOffset);
+                const int row0 = static_cast<int>(my_rank) * rows_per;
+                constexpr int kGroups = kBN / 8;                       // 8 columns = one 16-byte store
+                const int tid = (warp - kEpiWarp0) * 32 + lane;        // 0..127
+                for (int e = tid; e < my_rows * kGroups; e += 128) {
+                    const int rr = e / kGroups, c8 = e - rr * kGroups;
+                    float acc8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+                    for (int src = 0; src < split; ++src) {
+                        const float *rowp = src == static_cast<int>(my_rank)
+                                                ? own + (row0 + rr) * L::kRecvStride
+                                                : recv + (src * rows_per + rr) * L::kRecvStride;
+                        const float4 a = *reinterpret_cast<const float4 *>(rowp + 8 * c8);
+                        const float4 b = *reinterpret_cast<const float4 *>(rowp + 8 * c8 + 4);
+                        acc8[0] += a.x; acc8[1] += a.y; acc8[2] += a.z; acc8[3] += a.w;
+                        acc8[4] += b.x; acc8[5] += b.y; acc8[6] += b.z; acc8[7] += b.w;
+                    }
+                    const int col = tl.n0 + 8 * c8;
+                    const int tok = tl.tok0 + row0 + rr;
+                    if (col < p.N && tok < tl.tok_end) {
+                        uint4 pk;
+                        __nv_bfloat162 h0 = __floats2bfloat162_rn(acc8[0], acc8[1]);
+                        __nv_bfloat162 h1 = __floats2bfloat162_rn(acc8[2], acc8[3]);
+                        __nv_bfloat162 h2 = __floats2bfloat162_rn(acc8[4], acc8[5]);
+                        __nv_bfloat162 h3 = __floats2bfloat162_rn(acc8[6], acc8[7]);
+                        pk.x = *reinterpret_cast<uint32_t *>(&h0);
+                        pk.y = *reinterpret_cast<uint32_t *>(&h1);
+                        pk.z = *reinterpret_cast<uint32_t *>(&h2);
+                        pk.w = *reinterpret_cast<uint32_t *>(&h3);
+                        *reinterpret_cast<uint4 *>(p.d + static_cast<size_t>(tok) * p.N + col) = pk;
+                    }
+                }
+            }
+        }
+    }
+    if (clustered) {
+        // warps outside the epilogue complete the set-up arrival here; then no
+        // CTA leaves while a peer's bulk copy may still read its staging or
+        // write its receive buffer
+        if (warp < kEpiWarp0) ptx::cluster_wait_acquire();
+        __syncwarp();
+        ptx::cluster_sync_all();
     }
 
     // ---------------------------------------------------------------- teardown

@@ -62,6 +62,28 @@ def test_dense_matches_oracle(M, N, K):
     compare(d, _ref(prob), np.ones(prob.d_shape(), bool))
 
 
+@pytest.mark.parametrize("M,N,K", [(100, 264, 1000), (128, 2112, 512), (33, 128, 4096), (64, 384, 256)])
+def test_dense_split_k_shapes(M, N, K):
+    """M <= 128 with few weight tiles: K split over a cluster of CTAs, partials
+    reduced through distributed shared memory (N tail, K tail, short K)."""
+    prob = W.make_bf16_dense(M, N, K, seed=M * 7 + N + K)
+    d = _run(prob).double().cpu().numpy()
+    compare(d, _ref(prob), np.ones(prob.d_shape(), bool))
+
+
+def test_dense_split_k_exact_integers():
+    """Integer operands: the split partial sums are exact in FP32, so the
+    rank-order reduction must give the exact result bit for bit."""
+    rng = np.random.default_rng(8)
+    M, N, K = 64, 256, 2048
+    ai, bi = rng.integers(-3, 4, size=(M, K)), rng.integers(-3, 4, size=(N, K))
+    prob = W.BF16Problem("dense", M, N, K, 1, W._bf16_bits(ai.astype(np.float32)),
+                         W._bf16_bits(bi.astype(np.float32))[None])
+    d = _run(prob).cpu()
+    exact = torch.from_numpy((ai @ bi.T).astype(np.float32)).to(torch.bfloat16)
+    assert torch.equal(d.view(torch.int16), exact.view(torch.int16))
+
+
 def test_dense_exact_integers():
     rng = np.random.default_rng(5)
     M, N, K = 200, 384, 320
