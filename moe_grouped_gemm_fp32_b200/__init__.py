@@ -1,4 +1,6 @@
-"""Python binding of the B200 FP8 block-scaled NT GEMM library (``_dg.so``).
+"""Python binding of the B200 GEMM library (``_dg.so``): FP8 block-scaled NT
+GEMMs (dense, M-grouped contiguous and masked, K-grouped), the fused expert
+FFN, BF16 GEMMs in the same layouts, and the per-token 1x128 quantiser.
 
 Argument marshalling only: every function below checks dtypes and shapes of
 torch CUDA tensors, reads their raw pointers and calls the C function of the
@@ -6,10 +8,10 @@ same name declared in ``include/dg.h``.  All arithmetic runs in the CUDA
 kernels of ``_dg.so``.  There is no fallback: if the shared library is missing
 or fails to load, importing the library handle raises.
 
-Storage formats (see ``include/dg.h``): A/B are uint8 E4M3 bytes, K-major;
-quantiser inputs are bfloat16 rows;
+Storage formats (see ``include/dg.h``): FP8 A/B are uint8 E4M3 bytes, K-major;
 sfa is float32 [KB, ld_sfa] ("MN-major"; [G, KB, ld_sfa] for the masked
-layout); sfb is float32 [G, NB, KB]; D is bfloat16.
+layout); sfb is float32 [G, NB, KB]; D is bfloat16.  BF16 GEMM operands and
+quantiser inputs are bfloat16 rows.
 """
 from __future__ import annotations
 
