@@ -90,3 +90,21 @@ def test_python_binding_rejects_cpu_tensors():
     with pytest.raises(TypeError):
         dg.dg_fp8_gemm_nt(a, torch.zeros((1, 64)), torch.zeros((128, 128), dtype=torch.uint8),
                           torch.zeros((1, 1)), torch.zeros((64, 128), dtype=torch.bfloat16))
+
+
+def test_header_is_plain_c_and_links(tmp_path):
+    """include/dg.h compiles as C11 (no C++ in the signatures) and every
+    function it declares links against _dg.so."""
+    dg_build.build()
+    names = dg.exported_names()
+    src = tmp_path / "use_dg.c"
+    body = "\n".join(f"    (void)&{n};" for n in names)
+    src.write_text('#include "dg.h"\nint main(void) {\n' + body + "\n    return 0;\n}\n")
+    import os
+    inc = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include")
+    lib_dir = os.path.dirname(dg.LIB_PATH)
+    exe = tmp_path / "use_dg"
+    r = subprocess.run(["gcc", "-std=c11", "-Wall", "-Werror", "-I", inc, str(src), "-o", str(exe),
+                        os.path.join(lib_dir, "_dg.so"), "-Wl,-rpath," + lib_dir],
+                       capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
