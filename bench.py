@@ -9,7 +9,9 @@ workloads time the per-token 1x128 activation quantiser that produces the
 GEMM's A operand instead (GB/s of BF16 in + E4M3 and scales out).  L2 is flushed
 before every timed step (a 512 MB write, then a 256 MB read so that no dirty
 line of the flush is left to write back during the step) and the step is
-timed alone with CUDA events on the launching stream.  Multi-GPU (torchrun): each rank runs its own
+timed alone with CUDA events on the launching stream.  The masked GEMM
+workloads are also timed as 50 calls replayed from one CUDA graph (key
+``graph``).  Multi-GPU (torchrun): each rank runs its own
 independent problem (no collective on the data path, weak scaling); the step
 time is the max over ranks.  ``--impl reference`` times the CPU oracle (FP64,
 all host cores) on a bounded sample of the same workload instead.
@@ -55,6 +57,9 @@ KERNEL_SOURCES = {
                          "moe_grouped_gemm_fp32_b200/csrc/ptx.cuh"],
 }
 FLUSH_BYTES = 512 << 20
+# masked decode calls are also timed replayed from one CUDA graph of this many
+# back-to-back launches (the masked layout exists so that decode can be captured)
+GRAPH_CALLS = 50
 
 
 def is_quant(workload: str) -> bool:
@@ -407,8 +412,43 @@ def run_ours(args, rank, world, local_rank):
     h2d = sum(v.numel() * v.element_size() for v in host.values())
     d2h = op.d2h_bytes()
 
-    ms, e2e_ms = max_over_ranks([ms, e2e_ms], dev, world)
-    return prob, ms, e2e_ms, h2d, d2h, clocks
+    graph_ms = (graph_timing(op, devt, dev, stream)
+                if prob.layout == "masked" and not is_quant(args.workload) else 0.0)
+    status = dg.dg_get_device_status(clear=True)
+    if status:
+        raise RuntimeError(f"kernel status word {status:#x}")
+
+    ms, e2e_ms, graph_ms = max_over_ranks([ms, e2e_ms, graph_ms], dev, world)
+    return prob, ms, e2e_ms, h2d, d2h, clocks, graph_ms
+
+
+def graph_timing(op, devt, dev, stream, replays: int = 5) -> float:
+    """Milliseconds per call with GRAPH_CALLS calls captured in one CUDA graph and
+    replayed back to back (median of ``replays`` replays).  No L2 flush between
+    the calls: the masked workloads' B operand alone is larger than L2, so B
+    still streams from HBM on every call while A may stay in L2."""
+    import torch
+    side = torch.cuda.Stream(dev)
+    side.wait_stream(stream)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=side):
+        for _ in range(GRAPH_CALLS):
+            op.call(devt, side)
+    stream.wait_stream(side)
+    g.replay()
+    torch.cuda.synchronize(dev)
+    times = []
+    for _ in range(replays):
+        st = torch.cuda.Event(enable_timing=True)
+        en = torch.cuda.Event(enable_timing=True)
+        st.record(stream)
+        g.replay()
+        en.record(stream)
+        torch.cuda.synchronize(dev)
+        times.append(st.elapsed_time(en) / GRAPH_CALLS)
+    del g
+    torch.cuda.synchronize(dev)
+    return statistics.median(times)
 
 
 def metric_value(prob, unit, ms, world):
@@ -661,7 +701,7 @@ def main():
         dist.init_process_group("nccl", timeout=timedelta(seconds=300),
                                 device_id=torch.device("cuda", local_rank))
     try:
-        prob, ms, e2e_ms, h2d, d2h, clocks = run_ours(args, rank, world, local_rank)
+        prob, ms, e2e_ms, h2d, d2h, clocks, graph_ms = run_ours(args, rank, world, local_rank)
     finally:
         if world > 1:
             dist.destroy_process_group()
@@ -699,6 +739,10 @@ def main():
         "gpu_launches": args.steps,
         "clocks": clocks,
     }
+    if graph_ms > 0:
+        line["graph"] = {"value": metric_value(prob, unit, graph_ms, world), "unit": unit,
+                         "ms_per_call": graph_ms, "calls_per_graph": GRAPH_CALLS,
+                         "l2": "not flushed between calls (B alone exceeds L2)"}
     if not args.no_cpu_baseline and world == 1:
         cb = cpu_baseline(prob, unit)
         cb.pop("seconds_per_step", None)
