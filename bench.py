@@ -57,6 +57,9 @@ KERNEL_SOURCES = {
                          "moe_grouped_gemm_fp32_b200/csrc/ptx.cuh"],
 }
 FLUSH_BYTES = 512 << 20
+# B200 data-sheet figures, printed beside the measured denominators: HBM3e
+# GB/s (HGX B200) and dense (no 2:4 sparsity) tensor TFLOP/s
+NOMINAL_PEAK = {"hbm": 7700.0, "fp8": 4500.0, "bf16": 2250.0}
 # masked decode calls are also timed replayed from one CUDA graph of this many
 # back-to-back launches (the masked layout exists so that decode can be captured)
 GRAPH_CALLS = 50
@@ -388,6 +391,7 @@ def run_ours(args, rank, world, local_rank):
     clocks = sampler.stop()
     per_step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
     ms = sum(per_step_ms) / len(per_step_ms)
+    ms_median = statistics.median(per_step_ms)
     status = dg.dg_get_device_status(clear=True)
     if status:
         raise RuntimeError(f"kernel status word {status:#x}")
@@ -418,8 +422,8 @@ def run_ours(args, rank, world, local_rank):
     if status:
         raise RuntimeError(f"kernel status word {status:#x}")
 
-    ms, e2e_ms, graph_ms = max_over_ranks([ms, e2e_ms, graph_ms], dev, world)
-    return prob, ms, e2e_ms, h2d, d2h, clocks, graph_ms
+    ms, ms_median, e2e_ms, graph_ms = max_over_ranks([ms, ms_median, e2e_ms, graph_ms], dev, world)
+    return prob, ms, ms_median, e2e_ms, h2d, d2h, clocks, graph_ms
 
 
 def graph_timing(op, devt, dev, stream, replays: int = 5) -> float:
@@ -701,7 +705,7 @@ def main():
         dist.init_process_group("nccl", timeout=timedelta(seconds=300),
                                 device_id=torch.device("cuda", local_rank))
     try:
-        prob, ms, e2e_ms, h2d, d2h, clocks, graph_ms = run_ours(args, rank, world, local_rank)
+        prob, ms, ms_median, e2e_ms, h2d, d2h, clocks, graph_ms = run_ours(args, rank, world, local_rank)
     finally:
         if world > 1:
             dist.destroy_process_group()
@@ -712,11 +716,13 @@ def main():
     peaks, peak_src = measured_peaks()
     if unit == "GB/s":
         bound, peak, runit = "hbm", peaks["hbm_gbs"], "GB/s"
+        nominal = NOMINAL_PEAK["hbm"]
         achieved = prob.bytes() / (ms * 1e-3) / 1e9
     else:
         bound, runit = "tensor", "TFLOP/s"
         # BF16: the measured BF16 peak; FP8 dense = 2 x BF16 dense (nominal ratio)
         peak = peaks["bf16_tflops"] * (1.0 if is_bf16(args.workload) else 2.0)
+        nominal = NOMINAL_PEAK["bf16" if is_bf16(args.workload) else "fp8"]
         achieved = prob.flops() / (ms * 1e-3) / 1e12
     pages = PAGES_NUMBER.get(args.workload)
     line = {
@@ -730,9 +736,10 @@ def main():
         "config": {"workload": args.workload, **shape_config(prob),
                    "l2": "flushed before every step (512 MB write, then 256 MB read)",
                    **({} if is_quant(args.workload) else {"tflops": prob.flops() / (ms * 1e-3) / 1e12}),
-                   "gbps": prob.bytes() / (ms * 1e-3) / 1e9},
+                   "gbps": prob.bytes() / (ms * 1e-3) / 1e9, "ms_median_step": ms_median},
         "roofline": {"bound": bound, "achieved": achieved, "peak": peak, "unit": runit,
                      "frac": achieved / peak, "traffic": profiled_traffic(args.workload),
+                     "nominal_peak": nominal, "frac_of_nominal": achieved / nominal,
                      "peak_source": f"{peak_src} ({'hbm_gbs' if bound == 'hbm' else 'bf16_tflops' if is_bf16(args.workload) else '2 x bf16_tflops'})"},
         "e2e": {"value": metric_value(prob, unit, e2e_ms, world), "unit": unit,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
