@@ -117,6 +117,13 @@ def test_masked_matches_oracle_and_leaves_rows(masked_m, Mmax, N, K):
     assert (bits[~valid] == np.int16(SENTINEL)).all(), "rows past masked_m were written"
 
 
+def test_masked_maximum_group_count():
+    """G = 1024, the masked call's largest group count; every seventh group empty."""
+    counts = np.random.default_rng(1024).integers(0, 65, size=1024)
+    counts[::7] = 0
+    test_masked_matches_oracle_and_leaves_rows(counts.tolist(), 64, 128, 128)
+
+
 def test_masked_graph_replay_with_new_counts():
     prob = W.make_bf16_masked([40, 0, 128], 128, 256, 384, seed=9)
     a, b = _t(prob.a), _t(prob.b)

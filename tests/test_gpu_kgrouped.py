@@ -57,6 +57,18 @@ def test_k_grouped_matches_oracle(ks, M, N):
             assert (d[g] == 0).all(), f"empty group {g} not zero"
 
 
+def test_k_grouped_maximum_group_count():
+    """G = 1024 groups along K (the prefix table's capacity), about three in
+    four of them empty: empty groups give zeros, the others their own K range."""
+    rng = np.random.default_rng(4096)
+    ks = np.where(rng.random(1024) < 0.25, 128, 0).astype(np.int32)
+    ks[-1] = 256
+    prob = W.make_k_grouped(ks, 128, 128, seed=4097)
+    dp, d = _run(prob)
+    compare(d, oracle.solve(prob), valid_mask(prob))
+    assert (d[ks == 0] == 0).all()
+
+
 def test_k_grouped_exact_integers():
     """Integer operands in {-1, 0, 1} with power-of-two scales: every partial
     sum and the BF16 output are exact, so D must match bit for bit."""

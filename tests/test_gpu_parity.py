@@ -177,6 +177,21 @@ def test_masked_rows_untouched(masked_m, Mmax):
         assert (raw[g, :m] != np.int16(SENTINEL)).all()
 
 
+def test_masked_maximum_group_count():
+    """G = 1024, the largest group count the masked call accepts (its tile table
+    holds one prefix entry per group plus the total): mostly tiny groups, every
+    seventh one empty, the last one full."""
+    rng = np.random.default_rng(1024)
+    masked_m = rng.integers(0, 65, size=1024)
+    masked_m[::7] = 0
+    masked_m[-1] = 64
+    prob = W.make_masked(masked_m.tolist(), 64, 128, 256, seed=1025)
+    dp, d, ref, _ = _run_full(prob, sentinel=True)
+    raw = dp.d.view(torch.int16).cpu().numpy()
+    for g, m in enumerate(masked_m):
+        assert (raw[g, m:] == np.int16(SENTINEL)).all(), f"group {g} rows >= {m} written"
+
+
 def test_masked_n_tail_large_k():
     _run_full(W.make_masked([200, 33, 0, 256], 256, 2112, 2048, seed=21))
 

@@ -187,6 +187,16 @@ def test_masked_matches_oracle(masked_m, Mmax, K):
     _check_masked(prob, q, sfa)
 
 
+def test_masked_maximum_group_count():
+    """G = 1024, the largest group count of the masked quantiser (its row-prefix
+    table has one entry per group plus the total); every seventh group empty."""
+    counts = np.random.default_rng(1023).integers(0, 17, size=1024)
+    counts[::7] = 0
+    prob = W.make_activations_masked(counts.tolist(), 16, 256, seed=1023)
+    q, sfa = _quant_masked(prob)
+    _check_masked(prob, q, sfa)
+
+
 def test_masked_graph_replay():
     prob = W.make_activations_masked([17, 0, 64, 33], 64, 512, seed=41)
     q, sfa = _quant_masked(prob, graph=True)
