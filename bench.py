@@ -212,6 +212,8 @@ def max_over_ranks(values, device, world: int):
 class GemmCall:
     """Pinned host inputs, device output and the library call of one GEMM problem."""
 
+    launches_per_step = 1
+
     def __init__(self, prob, dev):
         import numpy as np
         import torch
@@ -251,6 +253,8 @@ class GemmCall:
 class Bf16Call:
     """Pinned BF16 operands, device output and the library call of one BF16 GEMM."""
 
+    launches_per_step = 1
+
     def __init__(self, prob, dev):
         import numpy as np
         import torch
@@ -284,6 +288,8 @@ class FFNCall:
     """Pinned tokens and expert weights, device intermediate and output, and the
     fused expert FFN call (two launches: GEMM1 + SwiGLU + requantisation, GEMM2)."""
 
+    launches_per_step = 2
+
     def __init__(self, prob, dev):
         import numpy as np
         import torch
@@ -310,6 +316,8 @@ class FFNCall:
 
 class QuantCall:
     """Pinned BF16 activations, device codes and scales, and the quantiser call."""
+
+    launches_per_step = 1
 
     def __init__(self, prob, dev):
         import torch
@@ -423,7 +431,7 @@ def run_ours(args, rank, world, local_rank):
         raise RuntimeError(f"kernel status word {status:#x}")
 
     ms, ms_median, e2e_ms, graph_ms = max_over_ranks([ms, ms_median, e2e_ms, graph_ms], dev, world)
-    return prob, ms, ms_median, e2e_ms, h2d, d2h, clocks, graph_ms
+    return prob, ms, ms_median, e2e_ms, h2d, d2h, clocks, graph_ms, op.launches_per_step
 
 
 def graph_timing(op, devt, dev, stream, replays: int = 5) -> float:
@@ -705,7 +713,7 @@ def main():
         dist.init_process_group("nccl", timeout=timedelta(seconds=300),
                                 device_id=torch.device("cuda", local_rank))
     try:
-        prob, ms, ms_median, e2e_ms, h2d, d2h, clocks, graph_ms = run_ours(args, rank, world, local_rank)
+        prob, ms, ms_median, e2e_ms, h2d, d2h, clocks, graph_ms, launches = run_ours(args, rank, world, local_rank)
     finally:
         if world > 1:
             dist.destroy_process_group()
@@ -743,7 +751,7 @@ def main():
                      "peak_source": f"{peak_src} ({'hbm_gbs' if bound == 'hbm' else 'bf16_tflops' if is_bf16(args.workload) else '2 x bf16_tflops'})"},
         "e2e": {"value": metric_value(prob, unit, e2e_ms, world), "unit": unit,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": args.steps,
+        "gpu_launches": args.steps * launches,
         "clocks": clocks,
     }
     if graph_ms > 0:
