@@ -118,6 +118,44 @@ def _req(t, dtype, name, ndim=None):
     return t.data_ptr()
 
 
+def _shape(t, want, name):
+    """Raise ValueError unless ``t`` has exactly the shape ``want``; a None
+    entry is a size this call cannot know (left to the C call's own checks).
+    The C functions receive only pointers and sizes, so a buffer smaller than
+    its sizes imply must be caught here."""
+    got = tuple(t.shape)
+    if len(got) != len(want) or any(w is not None and g != w for g, w in zip(got, want)):
+        shown = tuple("*" if w is None else w for w in want)
+        raise ValueError(f"{name} has shape {got}, expected {shown}")
+
+
+def _blocks(n):
+    """Number of 128-wide blocks of a size that must be a multiple of 128
+    (None otherwise: the C call rejects such a size itself)."""
+    return n // 128 if n % 128 == 0 else None
+
+
+def _ceil_blocks(n):
+    return (n + 127) // 128
+
+
+def _call(where, fn, tensors, stream, *args):
+    """Call ``fn(*args, stream_handle)`` and raise on a non-success status.
+    The C library launches on the current CUDA device, so every tensor (and
+    the stream, if given) must live on that device."""
+    import torch
+    devs = {t.device for t in tensors}
+    if len(devs) != 1:
+        raise ValueError(f"{where}: all tensors must be on one CUDA device, got {sorted(map(str, devs))}")
+    dev = devs.pop()
+    if dev.type == "cuda" and dev.index != torch.cuda.current_device():
+        raise ValueError(f"{where}: tensors are on {dev} but the current device is "
+                         f"cuda:{torch.cuda.current_device()} (select it with torch.cuda.device)")
+    if stream is not None and stream.device != dev:
+        raise ValueError(f"{where}: stream is on {stream.device}, tensors on {dev}")
+    _check(fn(*args, _stream_handle(stream)), where)
+
+
 # --------------------------------------------------------------------------- GEMMs
 def dg_fp8_gemm_nt(a, sfa, b, sfb, d, stream=None):
     """D[M,N] (bf16) = block-scaled A[M,K] * B[N,K]^T.
@@ -125,13 +163,19 @@ def dg_fp8_gemm_nt(a, sfa, b, sfb, d, stream=None):
     a uint8 [M,K]; sfa float32 [KB, ld_sfa]; b uint8 [N,K] (or [1,N,K]);
     sfb float32 [NB,KB] (or [1,NB,KB]); d bfloat16 [M,N]."""
     import torch
+    ptrs = (_req(a, torch.uint8, "a", 2), _req(sfa, torch.float32, "sfa", 2),
+            _req(b, torch.uint8, "b", (2, 3)), _req(sfb, torch.float32, "sfb", (2, 3)),
+            _req(d, torch.bfloat16, "d", 2))
     M, K = a.shape
     N = b.shape[-2]
     ld = sfa.shape[-1]
-    st = lib().dg_fp8_gemm_nt(_req(a, torch.uint8, "a", 2), _req(sfa, torch.float32, "sfa", 2), ld,
-                              _req(b, torch.uint8, "b", (2, 3)), _req(sfb, torch.float32, "sfb", (2, 3)),
-                              _req(d, torch.bfloat16, "d", 2), M, N, K, _stream_handle(stream))
-    _check(st, "dg_fp8_gemm_nt")
+    KB = _blocks(K)
+    _shape(b, (1,) * (b.dim() - 2) + (N, K), "b")
+    _shape(sfa, (KB, ld), "sfa")
+    _shape(sfb, (1,) * (sfb.dim() - 2) + (_ceil_blocks(N), KB), "sfb")
+    _shape(d, (M, N), "d")
+    _call("dg_fp8_gemm_nt", lib().dg_fp8_gemm_nt, (a, sfa, b, sfb, d), stream,
+          ptrs[0], ptrs[1], ld, ptrs[2], ptrs[3], ptrs[4], M, N, K)
     return d
 
 
@@ -139,14 +183,20 @@ def dg_m_grouped_fp8_gemm_nt_contiguous(a, sfa, b, sfb, d, m_indices, stream=Non
     """Contiguous M-grouped GEMM.  a uint8 [M_total,K]; b uint8 [G,N,K];
     sfb float32 [G,NB,KB]; d bfloat16 [M_total,N]; m_indices int32 [M_total]."""
     import torch
+    ptrs = (_req(a, torch.uint8, "a", 2), _req(sfa, torch.float32, "sfa", 2),
+            _req(b, torch.uint8, "b", 3), _req(sfb, torch.float32, "sfb", 3),
+            _req(d, torch.bfloat16, "d", 2), _req(m_indices, torch.int32, "m_indices", 1))
     M_total, K = a.shape
     G, N, _ = b.shape
-    st = lib().dg_m_grouped_fp8_gemm_nt_contiguous(
-        _req(a, torch.uint8, "a", 2), _req(sfa, torch.float32, "sfa", 2), sfa.shape[-1],
-        _req(b, torch.uint8, "b", 3), _req(sfb, torch.float32, "sfb", 3),
-        _req(d, torch.bfloat16, "d", 2), _req(m_indices, torch.int32, "m_indices", 1),
-        M_total, N, K, G, _stream_handle(stream))
-    _check(st, "dg_m_grouped_fp8_gemm_nt_contiguous")
+    KB = _blocks(K)
+    _shape(b, (G, N, K), "b")
+    _shape(sfa, (KB, None), "sfa")
+    _shape(sfb, (G, _ceil_blocks(N), KB), "sfb")
+    _shape(d, (M_total, N), "d")
+    _shape(m_indices, (M_total,), "m_indices")
+    _call("dg_m_grouped_fp8_gemm_nt_contiguous", lib().dg_m_grouped_fp8_gemm_nt_contiguous,
+          (a, sfa, b, sfb, d, m_indices), stream,
+          ptrs[0], ptrs[1], sfa.shape[-1], ptrs[2], ptrs[3], ptrs[4], ptrs[5], M_total, N, K, G)
     return d
 
 
@@ -155,14 +205,20 @@ def dg_m_grouped_fp8_gemm_nt_masked(a, sfa, b, sfb, d, masked_m, stream=None):
     b uint8 [G,N,K]; sfb float32 [G,NB,KB]; d bfloat16 [G,Mmax,N];
     masked_m int32 [G] (device).  Rows >= masked_m[g] of d are not written."""
     import torch
+    ptrs = (_req(a, torch.uint8, "a", 3), _req(sfa, torch.float32, "sfa", 3),
+            _req(b, torch.uint8, "b", 3), _req(sfb, torch.float32, "sfb", 3),
+            _req(d, torch.bfloat16, "d", 3), _req(masked_m, torch.int32, "masked_m", 1))
     G, Mmax, K = a.shape
     N = b.shape[1]
-    st = lib().dg_m_grouped_fp8_gemm_nt_masked(
-        _req(a, torch.uint8, "a", 3), _req(sfa, torch.float32, "sfa", 3), sfa.shape[-1],
-        _req(b, torch.uint8, "b", 3), _req(sfb, torch.float32, "sfb", 3),
-        _req(d, torch.bfloat16, "d", 3), _req(masked_m, torch.int32, "masked_m", 1),
-        G, Mmax, N, K, _stream_handle(stream))
-    _check(st, "dg_m_grouped_fp8_gemm_nt_masked")
+    KB = _blocks(K)
+    _shape(b, (G, N, K), "b")
+    _shape(sfa, (G, KB, None), "sfa")
+    _shape(sfb, (G, _ceil_blocks(N), KB), "sfb")
+    _shape(d, (G, Mmax, N), "d")
+    _shape(masked_m, (G,), "masked_m")
+    _call("dg_m_grouped_fp8_gemm_nt_masked", lib().dg_m_grouped_fp8_gemm_nt_masked,
+          (a, sfa, b, sfb, d, masked_m), stream,
+          ptrs[0], ptrs[1], sfa.shape[-1], ptrs[2], ptrs[3], ptrs[4], ptrs[5], G, Mmax, N, K)
     return d
 
 
@@ -172,17 +228,20 @@ def dg_k_grouped_fp8_gemm_nt_contiguous(a, sfa, b, sfb, d, ks, stream=None):
     [KB, ld_sfa]; b uint8 [N,K]; sfb float32 [NB,KB]; d bfloat16 [G,M,N];
     ks int32 [G] (device), multiples of 128 adding up to K."""
     import torch
+    ptrs = (_req(a, torch.uint8, "a", 2), _req(sfa, torch.float32, "sfa", 2),
+            _req(b, torch.uint8, "b", (2, 3)), _req(sfb, torch.float32, "sfb", (2, 3)),
+            _req(d, torch.bfloat16, "d", 3), _req(ks, torch.int32, "ks", 1))
     M, K = a.shape
     N = b.shape[-2]
     G = ks.shape[0]
-    if tuple(d.shape) != (G, M, N):
-        raise ValueError(f"d must be [G, M, N] = {(G, M, N)}")
-    st = lib().dg_k_grouped_fp8_gemm_nt_contiguous(
-        _req(a, torch.uint8, "a", 2), _req(sfa, torch.float32, "sfa", 2), sfa.shape[-1],
-        _req(b, torch.uint8, "b", (2, 3)), _req(sfb, torch.float32, "sfb", (2, 3)),
-        _req(d, torch.bfloat16, "d", 3), _req(ks, torch.int32, "ks", 1), G, M, N, K,
-        _stream_handle(stream))
-    _check(st, "dg_k_grouped_fp8_gemm_nt_contiguous")
+    KB = _blocks(K)
+    _shape(b, (1,) * (b.dim() - 2) + (N, K), "b")
+    _shape(sfa, (KB, None), "sfa")
+    _shape(sfb, (1,) * (sfb.dim() - 2) + (_ceil_blocks(N), KB), "sfb")
+    _shape(d, (G, M, N), "d")
+    _call("dg_k_grouped_fp8_gemm_nt_contiguous", lib().dg_k_grouped_fp8_gemm_nt_contiguous,
+          (a, sfa, b, sfb, d, ks), stream,
+          ptrs[0], ptrs[1], sfa.shape[-1], ptrs[2], ptrs[3], ptrs[4], ptrs[5], G, M, N, K)
     return d
 
 
@@ -193,14 +252,25 @@ def dg_m_grouped_fp8_gemm_swiglu_quant_contiguous(a, sfa, b, sfb, q_out, s_out, 
     (interleaved per 128 rows) whose epilogue writes E4M3 codes q_out
     [M_total, I] and scales s_out [I/128, ld] of silu(gate) * up."""
     import torch
+    ptrs = (_req(a, torch.uint8, "a", 2), _req(sfa, torch.float32, "sfa", 2),
+            _req(b, torch.uint8, "b", 3), _req(sfb, torch.float32, "sfb", 3),
+            _req(q_out, torch.uint8, "q_out", 2), _req(s_out, torch.float32, "s_out", 2),
+            _req(m_indices, torch.int32, "m_indices", 1))
     M_total, K = a.shape
     G, N, _ = b.shape
-    st = lib().dg_m_grouped_fp8_gemm_swiglu_quant_contiguous(
-        _req(a, torch.uint8, "a", 2), _req(sfa, torch.float32, "sfa", 2), sfa.shape[-1],
-        _req(b, torch.uint8, "b", 3), _req(sfb, torch.float32, "sfb", 3),
-        _req(q_out, torch.uint8, "q_out", 2), _req(s_out, torch.float32, "s_out", 2), s_out.shape[-1],
-        _req(m_indices, torch.int32, "m_indices", 1), M_total, N, K, G, _stream_handle(stream))
-    _check(st, "dg_m_grouped_fp8_gemm_swiglu_quant_contiguous")
+    KB = _blocks(K)
+    I = N // 2 if N % 2 == 0 else None
+    _shape(b, (G, N, K), "b")
+    _shape(sfa, (KB, None), "sfa")
+    _shape(sfb, (G, _ceil_blocks(N), KB), "sfb")
+    _shape(q_out, (M_total, I), "q_out")
+    _shape(s_out, (_blocks(I) if I is not None else None, None), "s_out")
+    _shape(m_indices, (M_total,), "m_indices")
+    _call("dg_m_grouped_fp8_gemm_swiglu_quant_contiguous",
+          lib().dg_m_grouped_fp8_gemm_swiglu_quant_contiguous,
+          (a, sfa, b, sfb, q_out, s_out, m_indices), stream,
+          ptrs[0], ptrs[1], sfa.shape[-1], ptrs[2], ptrs[3], ptrs[4], ptrs[5], s_out.shape[-1],
+          ptrs[6], M_total, N, K, G)
     return q_out, s_out
 
 
@@ -209,51 +279,71 @@ def dg_m_grouped_fp8_ffn_contiguous(a, sfa, w1, sfb1, w2, sfb2, q_mid, s_mid, y,
     [M_total, H], w1 [G, 2I, H] (gate/up interleaved per 128 rows), w2 [G, H, I];
     q_mid [M_total, I] / s_mid [I/128, ld] are the caller's intermediate buffers."""
     import torch
+    ptrs = (_req(a, torch.uint8, "a", 2), _req(sfa, torch.float32, "sfa", 2),
+            _req(w1, torch.uint8, "w1", 3), _req(sfb1, torch.float32, "sfb1", 3),
+            _req(w2, torch.uint8, "w2", 3), _req(sfb2, torch.float32, "sfb2", 3),
+            _req(q_mid, torch.uint8, "q_mid", 2), _req(s_mid, torch.float32, "s_mid", 2),
+            _req(y, torch.bfloat16, "y", 2), _req(m_indices, torch.int32, "m_indices", 1))
     M_total, H = a.shape
     G, I2, _ = w1.shape
-    st = lib().dg_m_grouped_fp8_ffn_contiguous(
-        _req(a, torch.uint8, "a", 2), _req(sfa, torch.float32, "sfa", 2), sfa.shape[-1],
-        _req(w1, torch.uint8, "w1", 3), _req(sfb1, torch.float32, "sfb1", 3),
-        _req(w2, torch.uint8, "w2", 3), _req(sfb2, torch.float32, "sfb2", 3),
-        _req(q_mid, torch.uint8, "q_mid", 2), _req(s_mid, torch.float32, "s_mid", 2), s_mid.shape[-1],
-        _req(y, torch.bfloat16, "y", 2), _req(m_indices, torch.int32, "m_indices", 1),
-        M_total, H, I2 // 2, G, _stream_handle(stream))
-    _check(st, "dg_m_grouped_fp8_ffn_contiguous")
+    I = I2 // 2
+    HB, IB = _blocks(H), _blocks(I)
+    _shape(sfa, (HB, None), "sfa")
+    _shape(w1, (G, 2 * I, H), "w1")
+    _shape(sfb1, (G, _ceil_blocks(2 * I), HB), "sfb1")
+    _shape(w2, (G, H, I), "w2")
+    _shape(sfb2, (G, _ceil_blocks(H), IB), "sfb2")
+    _shape(q_mid, (M_total, I), "q_mid")
+    _shape(s_mid, (IB, None), "s_mid")
+    _shape(y, (M_total, H), "y")
+    _shape(m_indices, (M_total,), "m_indices")
+    _call("dg_m_grouped_fp8_ffn_contiguous", lib().dg_m_grouped_fp8_ffn_contiguous,
+          (a, sfa, w1, sfb1, w2, sfb2, q_mid, s_mid, y, m_indices), stream,
+          ptrs[0], ptrs[1], sfa.shape[-1], ptrs[2], ptrs[3], ptrs[4], ptrs[5], ptrs[6], ptrs[7],
+          s_mid.shape[-1], ptrs[8], ptrs[9], M_total, H, I, G)
     return y
 
 # --------------------------------------------------------------------------- BF16 GEMMs
 def dg_bf16_gemm_nt(a, b, d, stream=None):
     """D[M,N] = A[M,K] * B[N,K]^T, all bfloat16 (FP32 accumulation)."""
     import torch
+    ptrs = (_req(a, torch.bfloat16, "a", 2), _req(b, torch.bfloat16, "b", (2, 3)),
+            _req(d, torch.bfloat16, "d", 2))
     M, K = a.shape
     N = b.shape[-2]
-    st = lib().dg_bf16_gemm_nt(_req(a, torch.bfloat16, "a", 2), _req(b, torch.bfloat16, "b", (2, 3)),
-                               _req(d, torch.bfloat16, "d", 2), M, N, K, _stream_handle(stream))
-    _check(st, "dg_bf16_gemm_nt")
+    _shape(b, (1,) * (b.dim() - 2) + (N, K), "b")
+    _shape(d, (M, N), "d")
+    _call("dg_bf16_gemm_nt", lib().dg_bf16_gemm_nt, (a, b, d), stream, *ptrs, M, N, K)
     return d
 
 
 def dg_m_grouped_bf16_gemm_nt_contiguous(a, b, d, m_indices, stream=None):
     """Contiguous M-grouped BF16 GEMM: a [M_total,K], b [G,N,K], d [M_total,N]."""
     import torch
+    ptrs = (_req(a, torch.bfloat16, "a", 2), _req(b, torch.bfloat16, "b", 3),
+            _req(d, torch.bfloat16, "d", 2), _req(m_indices, torch.int32, "m_indices", 1))
     M_total, K = a.shape
     G, N, _ = b.shape
-    st = lib().dg_m_grouped_bf16_gemm_nt_contiguous(
-        _req(a, torch.bfloat16, "a", 2), _req(b, torch.bfloat16, "b", 3), _req(d, torch.bfloat16, "d", 2),
-        _req(m_indices, torch.int32, "m_indices", 1), M_total, N, K, G, _stream_handle(stream))
-    _check(st, "dg_m_grouped_bf16_gemm_nt_contiguous")
+    _shape(b, (G, N, K), "b")
+    _shape(d, (M_total, N), "d")
+    _shape(m_indices, (M_total,), "m_indices")
+    _call("dg_m_grouped_bf16_gemm_nt_contiguous", lib().dg_m_grouped_bf16_gemm_nt_contiguous,
+          (a, b, d, m_indices), stream, *ptrs, M_total, N, K, G)
     return d
 
 
 def dg_m_grouped_bf16_gemm_nt_masked(a, b, d, masked_m, stream=None):
     """Masked M-grouped BF16 GEMM: a [G,Mmax,K], b [G,N,K], d [G,Mmax,N]."""
     import torch
+    ptrs = (_req(a, torch.bfloat16, "a", 3), _req(b, torch.bfloat16, "b", 3),
+            _req(d, torch.bfloat16, "d", 3), _req(masked_m, torch.int32, "masked_m", 1))
     G, Mmax, K = a.shape
     N = b.shape[1]
-    st = lib().dg_m_grouped_bf16_gemm_nt_masked(
-        _req(a, torch.bfloat16, "a", 3), _req(b, torch.bfloat16, "b", 3), _req(d, torch.bfloat16, "d", 3),
-        _req(masked_m, torch.int32, "masked_m", 1), G, Mmax, N, K, _stream_handle(stream))
-    _check(st, "dg_m_grouped_bf16_gemm_nt_masked")
+    _shape(b, (G, N, K), "b")
+    _shape(d, (G, Mmax, N), "d")
+    _shape(masked_m, (G,), "masked_m")
+    _call("dg_m_grouped_bf16_gemm_nt_masked", lib().dg_m_grouped_bf16_gemm_nt_masked,
+          (a, b, d, masked_m), stream, *ptrs, G, Mmax, N, K)
     return d
 
 # --------------------------------------------------------------------------- quantisers
@@ -261,13 +351,13 @@ def dg_per_token_cast_to_fp8(x, q, sfa, stream=None):
     """Per-token 1x128 quantisation.  x bfloat16 [M,K]; q uint8 [M,K];
     sfa float32 [KB, ld_sfa] with ld_sfa >= M, a multiple of 4."""
     import torch
+    ptrs = (_req(x, torch.bfloat16, "x", 2), _req(q, torch.uint8, "q", 2),
+            _req(sfa, torch.float32, "sfa", 2))
     M, K = x.shape
-    if tuple(q.shape) != (M, K):
-        raise ValueError("q must have the shape of x")
-    st = lib().dg_per_token_cast_to_fp8(_req(x, torch.bfloat16, "x", 2), _req(q, torch.uint8, "q", 2),
-                                        _req(sfa, torch.float32, "sfa", 2), sfa.shape[-1], M, K,
-                                        _stream_handle(stream))
-    _check(st, "dg_per_token_cast_to_fp8")
+    _shape(q, (M, K), "q")
+    _shape(sfa, (_blocks(K), None), "sfa")
+    _call("dg_per_token_cast_to_fp8", lib().dg_per_token_cast_to_fp8, (x, q, sfa), stream,
+          *ptrs, sfa.shape[-1], M, K)
     return q, sfa
 
 
@@ -276,13 +366,14 @@ def dg_per_token_cast_to_fp8_masked(x, q, sfa, masked_m, stream=None):
     [G,Mmax,K]; sfa float32 [G,KB,ld_sfa]; masked_m int32 [G] (device).  Only
     rows < masked_m[g] are read and written."""
     import torch
+    ptrs = (_req(x, torch.bfloat16, "x", 3), _req(q, torch.uint8, "q", 3),
+            _req(sfa, torch.float32, "sfa", 3), _req(masked_m, torch.int32, "masked_m", 1))
     G, Mmax, K = x.shape
-    if tuple(q.shape) != (G, Mmax, K):
-        raise ValueError("q must have the shape of x")
-    st = lib().dg_per_token_cast_to_fp8_masked(
-        _req(x, torch.bfloat16, "x", 3), _req(q, torch.uint8, "q", 3), _req(sfa, torch.float32, "sfa", 3),
-        sfa.shape[-1], _req(masked_m, torch.int32, "masked_m", 1), G, Mmax, K, _stream_handle(stream))
-    _check(st, "dg_per_token_cast_to_fp8_masked")
+    _shape(q, (G, Mmax, K), "q")
+    _shape(sfa, (G, _blocks(K), None), "sfa")
+    _shape(masked_m, (G,), "masked_m")
+    _call("dg_per_token_cast_to_fp8_masked", lib().dg_per_token_cast_to_fp8_masked,
+          (x, q, sfa, masked_m), stream, ptrs[0], ptrs[1], ptrs[2], sfa.shape[-1], ptrs[3], G, Mmax, K)
     return q, sfa
 
 
