@@ -238,6 +238,28 @@ def test_masked_equals_dense_per_group():
         compare(to_f64(dd), ref, np.ones_like(ref, bool))
 
 
+def test_rejected_calls_leave_d_untouched():
+    """Argument errors are reported before anything is enqueued: each call
+    returns its status code and D keeps its sentinel bit for bit."""
+    prob = W.make_dense(64, 256, 512, seed=5)
+    dp = DeviceProblem(prob)
+    dp.fill_sentinel()
+    L = dg.lib()
+    a, sfa, b, sfb, d = (dp.a.data_ptr(), dp.sfa.data_ptr(), dp.b.data_ptr(), dp.sfb.data_ptr(),
+                         dp.d.data_ptr())
+    ld = prob.ld_sfa
+    assert L.dg_fp8_gemm_nt(a, sfa, ld, b, sfb, d, 64, 256, 500, None) == 3        # K % 128
+    assert L.dg_fp8_gemm_nt(a, sfa, ld, b, sfb, d, 64, 200, 512, None) == 3        # N % 16
+    assert L.dg_fp8_gemm_nt(a + 8, sfa, ld, b, sfb, d, 64, 256, 512, None) == 2    # misaligned A
+    assert L.dg_fp8_gemm_nt(a, sfa, ld + 2, b, sfb, d, 64, 256, 512, None) == 2    # ld_sfa % 4
+    assert L.dg_fp8_gemm_nt(None, sfa, ld, b, sfb, d, 64, 256, 512, None) == 1     # null A
+    mm = torch.zeros(1, dtype=torch.int32, device="cuda")
+    assert L.dg_m_grouped_fp8_gemm_nt_masked(a, sfa, ld, b, sfb, d, mm.data_ptr(), 1025, 64, 256,
+                                             512, None) == 3                           # G > 1024
+    torch.cuda.synchronize()
+    assert (dp.d.view(torch.int16) == SENTINEL).all(), "a rejected call wrote D"
+
+
 # ------------------------------------------------------------------ full-size workloads
 @pytest.mark.parametrize("name", ["dense_decode_m64", "dense_decode_m128"])
 def test_full_size_decode_full_oracle(name):
