@@ -119,3 +119,36 @@ def test_reference_arm_for_the_next_rows(workload):
     assert d["impl"] == "reference" and d["config"]["workload"] == workload
     assert d["value"] > 0 and d["unit"] == bench.UNIT[workload]
     assert d["cpu_baseline"]["kind"] == "oracle" and d["e2e"]["h2d_bytes_per_step"] == 0
+
+
+@pytest.mark.parametrize("workload,launches,graph", [("dense_decode_m64", 1, False), ("masked_g16", 1, True),
+                                                     ("ffn_g4", 2, False), ("quant_tokens_32768", 1, False)])
+def test_our_json_line_carries_every_contract_key(monkeypatch, capsys, workload, launches, graph):
+    """The line of our arm, assembled from a stubbed device run: every key the
+    bench contract names is present, with the roofline fraction, the launch
+    count and (masked GEMMs only) the CUDA-graph figure consistent."""
+    prob = bench.rank_problem(workload, 0)
+    clocks = {"sm_mhz": 1965, "sm_max_mhz": 1965, "reasons": []}
+    monkeypatch.setattr(bench, "run_ours",
+                        lambda args, rank, world, lr: (prob, 0.5, 0.49, 0.8, 100, 20, clocks,
+                                                       0.51 if graph else 0.0, launches))
+    monkeypatch.setattr(sys, "argv", ["bench.py", "--workload", workload, "--steps", "7", "--warmup", "3",
+                                      "--no-cpu-baseline"])
+    assert bench.main() == 0
+    out = [l for l in capsys.readouterr().out.splitlines() if l.strip()]
+    assert len(out) == 1
+    line = json.loads(out[0])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "scaling", "vs_baseline", "dtype", "data", "config", "roofline", "e2e", "gpu_launches",
+                "clocks"):
+        assert key in line, key
+    assert line["config"]["workload"] == workload and line["scaling"] == "weak"
+    roof = line["roofline"]
+    for key in ("bound", "achieved", "peak", "unit", "frac", "traffic"):
+        assert key in roof, key
+    assert abs(roof["frac"] - roof["achieved"] / roof["peak"]) < 1e-12
+    assert set(line["e2e"]) >= {"value", "unit", "h2d_bytes_per_step", "d2h_bytes_per_step"}
+    assert line["e2e"]["value"] < line["value"]          # the e2e step (0.8 ms) is slower than 0.5 ms
+    assert line["gpu_launches"] == 7 * launches
+    assert ("graph" in line) == graph
+    assert line["clocks"] == clocks
