@@ -106,8 +106,8 @@ DG_API dg_status_t dg_m_grouped_fp8_gemm_nt_contiguous(const uint8_t *a, const f
  * never written (bit-for-bit untouched).  Groups with masked_m[g] == 0 read
  * nothing.  A count outside [0, Mmax] is clamped and recorded as
  * DG_ERR_INVALID_VALUE in the device status word.  G <= 1024 and
- * G * Mmax < 2^31 (32-bit tensor-map row coordinates; a precondition, not
- * checked by the call -- a buffer that large would not fit in device memory).
+ * G * Mmax < 2^31 (32-bit tensor-map row coordinates), else
+ * DG_ERR_UNSUPPORTED_SHAPE.
  */
 DG_API dg_status_t dg_m_grouped_fp8_gemm_nt_masked(const uint8_t *a, const float *sfa, int ld_sfa,
                                             const uint8_t *b, const float *sfb,
@@ -129,9 +129,9 @@ DG_API dg_status_t dg_m_grouped_fp8_gemm_nt_masked(const uint8_t *a, const float
  *       multiple of 128, or a total other than K is recorded as
  *       DG_ERR_INVALID_VALUE in the device status word; the kernel then uses
  *       the K-blocks that exist (rounded down, clipped at K).
- * 1 <= G <= 1024; M == 0 is a no-op.  G * M < 2^31: the output's stacked
- * rows are addressed by 32-bit tensor-map coordinates (a precondition, not
- * checked by the call).
+ * 1 <= G <= 1024; M == 0 is a no-op.  G * M < 2^31 (the output's stacked
+ * rows are addressed by 32-bit tensor-map coordinates), else
+ * DG_ERR_UNSUPPORTED_SHAPE.
  */
 DG_API dg_status_t dg_k_grouped_fp8_gemm_nt_contiguous(const uint8_t *a, const float *sfa,
                                                        int ld_sfa, const uint8_t *b,
@@ -205,8 +205,8 @@ DG_API dg_status_t dg_m_grouped_bf16_gemm_nt_contiguous(const void *a, const voi
 
 /* Masked M-grouped BF16: a [G, Mmax, K], b [G, N, K], d [G, Mmax, N]; rows
  * m < masked_m[g] computed, the others never written (graph-compatible, as for
- * the FP8 masked call).  G <= 1024 and G * Mmax < 2^31 (as for the FP8
- * masked call: a precondition, not checked). */
+ * the FP8 masked call).  G <= 1024 and G * Mmax < 2^31, else
+ * DG_ERR_UNSUPPORTED_SHAPE (as for the FP8 masked call). */
 DG_API dg_status_t dg_m_grouped_bf16_gemm_nt_masked(const void *a, const void *b, void *d,
                                                     const int32_t *masked_m, int G, int Mmax,
                                                     int N, int K, void *stream);

@@ -205,6 +205,7 @@ dg_status_t dg_m_grouped_bf16_gemm_nt_masked(const void *a, const void *b, void 
     if (st != DG_SUCCESS) return st;
     if (!masked_m || G <= 0) return DG_ERR_INVALID_VALUE;
     if (G > dg::kMaxGroups) return DG_ERR_UNSUPPORTED_SHAPE;
+    if (static_cast<long long>(G) * Mmax > (1LL << 31) - 1) return DG_ERR_UNSUPPORTED_SHAPE;
     const DeviceInfo *info = nullptr;
     if ((st = device_info(&info)) != DG_SUCCESS) return st;
     if (Mmax == 0) return DG_SUCCESS;

@@ -463,6 +463,8 @@ dg_status_t dg_m_grouped_fp8_gemm_nt_masked(const uint8_t *a, const float *sfa, 
     if (st != DG_SUCCESS) return st;
     if (!masked_m || G <= 0) return DG_ERR_INVALID_VALUE;
     if (G > dg::kMaxGroups) return DG_ERR_UNSUPPORTED_SHAPE;
+    // the stacked [G * Mmax] rows of d are addressed by 32-bit tensor-map coordinates
+    if (static_cast<long long>(G) * Mmax > (1LL << 31) - 1) return DG_ERR_UNSUPPORTED_SHAPE;
     const DeviceInfo *info = nullptr;
     if ((st = device_info(&info)) != DG_SUCCESS) return st;
     if (Mmax == 0) return DG_SUCCESS;
@@ -514,6 +516,8 @@ dg_status_t dg_k_grouped_fp8_gemm_nt_contiguous(const uint8_t *a, const float *s
     if (st != DG_SUCCESS) return st;
     if (!ks || G <= 0) return DG_ERR_INVALID_VALUE;
     if (G > dg::kMaxGroups) return DG_ERR_UNSUPPORTED_SHAPE;
+    // the stacked [G * M] rows of d are addressed by 32-bit tensor-map coordinates
+    if (static_cast<long long>(G) * M > (1LL << 31) - 1) return DG_ERR_UNSUPPORTED_SHAPE;
     const DeviceInfo *info = nullptr;
     if ((st = device_info(&info)) != DG_SUCCESS) return st;
     if (M == 0) return DG_SUCCESS;

@@ -82,6 +82,11 @@ def test_grouped_validation(L):
     assert m(FAKE, FAKE, 256, FAKE, FAKE, FAKE, FAKE, 2000, 256, 256, 512, None) == 3  # G > 1024
     assert m(FAKE, FAKE, 128, FAKE, FAKE, FAKE, FAKE, 4, 256, 256, 512, None) == 1   # ld < Mmax
     assert m(FAKE, FAKE, 256, FAKE, FAKE, FAKE, FAKE, 4, 256, 256, 384, None) == 4   # no device
+    big = 1 << 21                                                                      # G * rows = 2^31
+    assert m(FAKE, FAKE, big, FAKE, FAKE, FAKE, FAKE, 1024, big, 256, 512, None) == 3
+    k = L.dg_k_grouped_fp8_gemm_nt_contiguous
+    assert k(FAKE, FAKE, big, FAKE, FAKE, FAKE, FAKE, 1024, big, 256, 512, None) == 3
+    assert L.dg_m_grouped_bf16_gemm_nt_masked(FAKE, FAKE, FAKE, FAKE, 1024, big, 256, 512, None) == 3
 
 
 def test_python_binding_rejects_cpu_tensors():
