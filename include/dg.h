@@ -31,7 +31,11 @@
  *     error nothing is launched and d is untouched.  DG_ERR_CUDA reports a
  *     failed launch or a CUDA runtime error (text via dg_last_cuda_error()).
  *     A kernel that gives up on a bounded wait records DG_ERR_TIMEOUT in the
- *     device status word (dg_get_device_status) instead of hanging.
+ *     device status word (dg_get_device_status) instead of hanging.  The call
+ *     that launched it has already returned DG_SUCCESS, and d may be partly
+ *     written.  The status word is one per device, shared by every call on
+ *     every stream: a caller that needs to know which call failed reads (and
+ *     clears) it between calls.
  *   - Thread safety: calls on different streams may run concurrently.
  */
 #ifndef DG_H_
@@ -86,6 +90,13 @@ DG_API dg_status_t dg_fp8_gemm_nt(const uint8_t *a, const float *sfa, int ld_sfa
  *             -1 is skipped).  Outputs of padding rows are unspecified (they
  *             may be written).  An index >= G makes the kernel skip the block
  *             and record DG_ERR_INVALID_VALUE in the device status word.
+ *             The layout packs each group's rows as one run of blocks; runs
+ *             may also repeat or alternate, within one limit: large calls
+ *             (N > 128, K >= 4096, G < 1024) compute 256-row block pairs,
+ *             and at most 1024 pairs may hold two different groups.  Past
+ *             that the excess pairs' second blocks are not written and
+ *             DG_ERR_INVALID_VALUE is recorded.  One run per group keeps the
+ *             count below G.
  * M_total % 128 == 0; M_total == 0 is a no-op.
  */
 DG_API dg_status_t dg_m_grouped_fp8_gemm_nt_contiguous(const uint8_t *a, const float *sfa, int ld_sfa,

@@ -6,6 +6,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cstdio>
 #include <cstdlib>
 
@@ -47,13 +48,14 @@ dg_status_t launch_bf16(const CUtensorMap &ma, const CUtensorMap &mb, const dg::
                         cudaStream_t stream, int grid_y = 1, int cluster_x = 1) {
     using L = dg::Bf16Smem<kBN, kStages, kSplitK>;
     auto kernel = dg::bf16_gemm_kernel<kBN, kStages, kLayout, kSplitK>;
-    static bool configured[kMaxDevices] = {};
+    // one-time per-device set-up (idempotent; the atomic flag keeps racing first calls defined)
+    static std::atomic<bool> configured[kMaxDevices] = {};
     int dev = 0;
     cudaGetDevice(&dev);
-    if (!configured[dev]) {
+    if (!configured[dev].load(std::memory_order_acquire)) {
         cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
         if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(bf16 smem)");
-        configured[dev] = true;
+        configured[dev].store(true, std::memory_order_release);
     }
     if (verbose())
         std::fprintf(stderr, "[dg] bf16_gemm layout=%d bn=%d stages=%d grid=%dx%d cluster=%d split=%d smem=%d\n",
@@ -95,11 +97,12 @@ template <int kBN, int kStages>
 int bf16_max_clusters(int split) {
     using L = dg::Bf16Smem<kBN, kStages, true>;
     auto kernel = dg::bf16_gemm_kernel<kBN, kStages, dg::kDense, true>;
-    static int cache[kMaxDevices][9] = {};
+    // per-device cache of an idempotent query (atomic: concurrent first calls are defined)
+    static std::atomic<int> cache[kMaxDevices][9] = {};
     int dev = 0;
     cudaGetDevice(&dev);
     if (split < 2 || split > 8) return 0;
-    if (cache[dev][split]) return cache[dev][split];
+    if (const int c = cache[dev][split].load(std::memory_order_relaxed)) return c;
     if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc) != cudaSuccess) {
         cudaGetLastError();
         return 0;
@@ -120,7 +123,7 @@ int bf16_max_clusters(int split) {
         cudaGetLastError();
         return 0;
     }
-    cache[dev][split] = n;
+    cache[dev][split].store(n, std::memory_order_relaxed);
     return n;
 }
 

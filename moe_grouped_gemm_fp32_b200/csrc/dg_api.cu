@@ -7,6 +7,7 @@
 
 #include <cstdio>
 #include <cstdlib>
+#include <atomic>
 #include <cstring>
 #include <mutex>
 
@@ -203,10 +204,12 @@ dg_status_t launch(const CUtensorMap &ma, const CUtensorMap &mb, const CUtensorM
                    int grid_x, int grid_y, int cluster_x, cudaStream_t stream) {
     using L = dg::SmemLayout<kBN, kSwap, kStages, kCtaGroup, kSwap && kLayout == dg::kDense && kBN <= 128>;
     auto kernel = dg::fp8_gemm_kernel<kBN, kSwap, kStages, kLayout, kCtaGroup, kSwiGLU>;
-    static bool attr_done[kMaxDevices] = {};
+    // one-time per-device set-up; it is idempotent, so two threads that race on
+    // the first call both do it and the atomic flag keeps the access defined
+    static std::atomic<bool> attr_done[kMaxDevices] = {};
     int dev = 0;
     cudaGetDevice(&dev);
-    if (!attr_done[dev]) {
+    if (!attr_done[dev].load(std::memory_order_acquire)) {
         cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              L::kAlloc);
         if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
@@ -224,7 +227,7 @@ dg_status_t launch(const CUtensorMap &ma, const CUtensorMap &mb, const CUtensorM
                 return DG_ERR_CUDA;
             }
         }
-        attr_done[dev] = true;
+        attr_done[dev].store(true, std::memory_order_release);
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid_x, grid_y, 1);
@@ -258,11 +261,12 @@ template <int kBN, bool kSwap, int kStages, int kLayout, int kCtaGroup = 1>
 int max_active_clusters(int cluster_x) {
     using L = dg::SmemLayout<kBN, kSwap, kStages, kCtaGroup, kSwap && kLayout == dg::kDense && kBN <= 128>;
     auto kernel = dg::fp8_gemm_kernel<kBN, kSwap, kStages, kLayout, kCtaGroup>;
-    static int cache[kMaxDevices][9] = {};
+    // per-device cache of an idempotent query (atomic: concurrent first calls are defined)
+    static std::atomic<int> cache[kMaxDevices][9] = {};
     int dev = 0;
     cudaGetDevice(&dev);
     if (cluster_x < 1 || cluster_x > 8) return 0;
-    if (cache[dev][cluster_x]) return cache[dev][cluster_x];
+    if (const int c = cache[dev][cluster_x].load(std::memory_order_relaxed)) return c;
     if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc) !=
         cudaSuccess) {
         cudaGetLastError();
@@ -284,7 +288,7 @@ int max_active_clusters(int cluster_x) {
         cudaGetLastError();
         return 0;
     }
-    cache[dev][cluster_x] = n;
+    cache[dev][cluster_x].store(n, std::memory_order_relaxed);
     return n;
 }
 

@@ -4,6 +4,7 @@
 // Nothing here synchronises the host or allocates memory.
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cstdio>
 
 #include "dg.h"
@@ -20,21 +21,24 @@ template <bool kMasked, bool kFastDiv>
 dg_status_t launch_quant(const dg::QuantParams &p, long long max_items, const DeviceInfo *info,
                          cudaStream_t stream) {
     auto kernel = dg::quant_1x128_kernel<kMasked, kFastDiv>;
-    static int occ[kMaxDevices] = {};
+    // per-device cache of an idempotent query (atomic: concurrent first calls are defined)
+    static std::atomic<int> occ[kMaxDevices] = {};
     int dev = 0;
     cudaGetDevice(&dev);
-    if (!occ[dev]) {
+    int resident = occ[dev].load(std::memory_order_relaxed);
+    if (!resident) {
         int n = 0;
         cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, dg::kQuantThreads, 0);
         if (e != cudaSuccess) return cuda_fail(e, "cudaOccupancyMaxActiveBlocksPerMultiprocessor");
-        occ[dev] = n > 0 ? n : 1;
+        resident = n > 0 ? n : 1;
+        occ[dev].store(resident, std::memory_order_relaxed);
     }
     const long long want = (max_items + dg::kQuantWarps - 1) / dg::kQuantWarps;
-    const long long full = static_cast<long long>(info->num_sms) * occ[dev];
+    const long long full = static_cast<long long>(info->num_sms) * resident;
     const int grid = static_cast<int>(want < full ? (want > 0 ? want : 1) : full);
     if (verbose())
         std::fprintf(stderr, "[dg] quant_1x128 masked=%d fast_div=%d grid=%d occ=%d\n", kMasked ? 1 : 0,
-                     kFastDiv ? 1 : 0, grid, occ[dev]);
+                     kFastDiv ? 1 : 0, grid, resident);
     kernel<<<grid, dg::kQuantThreads, 0, stream>>>(p);
     cudaError_t e = cudaGetLastError();
     return e == cudaSuccess ? DG_SUCCESS : cuda_fail(e, "quant_1x128_kernel launch");
