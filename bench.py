@@ -1,18 +1,27 @@
 """Benchmark of the FP8 block-scaled NT GEMM on B200.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                    [--shapes auto|none|NAME,NAME,...] [--impl ours|reference]
 
 One step = one call of the hot path (scheduling, TMA loads, tcgen05 MMA,
 per-K-block promotion, epilogue; swap-AB and split-K for small M) on one
-batch of seeded synthetic inputs already resident in HBM.  The ``quant_*``
-workloads time the per-token 1x128 activation quantiser that produces the
-GEMM's A operand instead (GB/s of BF16 in + E4M3 and scales out).  L2 is flushed
-before every timed step (a 512 MB write, then a 256 MB read so that no dirty
-line of the flush is left to write back during the step) and the step is
-timed alone with CUDA events on the launching stream.  The masked GEMM
+batch of seeded synthetic inputs already resident in HBM.  The headline
+workload is the largest configuration of the method's benchmark set, the
+M-grouped contiguous MoE-prefill GEMM (4 experts, 32768 tokens, N=4096,
+K=7168).  A default run then times every configuration of that set (dense
+128x256x512, dense decode M=64 and M=128 at N=2112 K=7168, dense
+4096x7168x16384, the contiguous prefill, masked decode with 16 experts) with
+the same steps, warm-up and L2 flush, and reports each under ``shapes`` with
+its roofline fraction.  The ``quant_*`` workloads time the per-token 1x128
+activation quantiser instead (GB/s of BF16 in + E4M3 and scales out).
+
+L2 is flushed before every timed step (a 512 MB write, then a 256 MB read so
+that no dirty line of the flush is left to write back during the step) and the
+step is timed alone with CUDA events on the launching stream.  The masked GEMM
 workloads are also timed as 50 calls replayed from one CUDA graph (key
-``graph``).  Multi-GPU (torchrun): each rank runs its own
-independent problem (no collective on the data path, weak scaling); the step
+``graph``).  SM clocks and throttle reasons are sampled through NVML while
+every timed region runs.  Multi-GPU (torchrun): each rank runs its own
+independent problem (no collective on the data path, weak scaling); every
 time is the max over ranks.  ``--impl reference`` times the CPU oracle (FP64,
 all host cores) on a bounded sample of the same workload instead.
 
@@ -21,10 +30,10 @@ Prints ONE JSON line on rank 0.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import hashlib
 import json
 import os
-import re
 import statistics
 import sys
 import threading
@@ -34,10 +43,21 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "FP8 TFLOPS and HBM GB/s per shape, % of B200 FP8/HBM roofline, 1 GPU"
-DEFAULT_WORKLOAD = "dense_decode_m64"
-# The pages' own figure for the exact same workload (H800, another machine:
+# the largest configuration of the benchmark set: the headline of every run
+DEFAULT_WORKLOAD = "contiguous_g4"
+# the configurations of the method's benchmark set (DeepGEMM page 2 "性能实测"
+# shapes plus the expert counts of the workload definitions), timed under
+# ``shapes`` in every default run
+SHAPES = ("dense_tiny", "dense_decode_m64", "dense_decode_m128", "dense_large", "contiguous_g4",
+          "masked_g16")
+# The pages' own figure for exactly the same workload (H800, another machine:
 # context only).  DeepGEMM page 2 "性能实测": M=64 N=2112 K=7168 -> 1688 GB/s.
+# The page's other rows leave one of M, N or K unstated, so no other workload
+# has an exact counterpart.
 PAGES_NUMBER = {"dense_decode_m64": (1688.0, "GB/s")}
+# DRAM bytes per launch from ncu captures, keyed by kernel and workload, each
+# with the hash of the kernel sources it was taken on
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
 UNIT = {"dense_tiny": "TFLOP/s", "dense_decode_m64": "GB/s", "dense_decode_m128": "GB/s",
         "dense_large": "TFLOP/s", "contiguous_g4": "TFLOP/s", "masked_g16": "GB/s",
         "kgrouped_g4": "TFLOP/s",
@@ -96,24 +116,25 @@ def measured_peaks():
 
 
 def profiled_traffic(workload: str):
-    """DRAM bytes per launch from the committed ncu summary of this workload,
-    or None when there is none or the kernel sources changed since."""
+    """DRAM bytes per launch (ncu ``dram__bytes_read.sum + dram__bytes_write.sum``)
+    of this workload's kernel from ``profiles/traffic.json``, or None when there
+    is no capture or the kernel sources changed since it was taken."""
     kernel = kernel_name(workload)
-    p = os.path.join(ROOT, "profiles", f"{kernel}_{workload}.md")
-    if not os.path.exists(p):
+    try:
+        with open(TRAFFIC_FILE) as fh:
+            entry = json.load(fh)["captures"][f"{kernel}/{workload}"]
+    except (OSError, KeyError, ValueError):
         return None
-    text = open(p).read()
-    m = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
-    h = re.search(r"kernel_source_hash:\s*([0-9a-f]+)", text)
-    if not m or not h or h.group(1) != kernel_source_hash(kernel):
+    if entry.get("kernel_source_hash") != kernel_source_hash(kernel):
         return None
-    return float(m.group(1))
+    return float(entry["dram_bytes_per_launch"])
 
 
 class ClockSampler:
-    """SM clock and throttle reasons of one GPU, read through NVML every few
-    milliseconds by a background thread while the timed region runs.  Reads
-    only; no setting of the GPU is touched."""
+    """SM clock and throttle reasons of one GPU, read through NVML every
+    millisecond by a background thread while a timed region runs (``resume`` /
+    ``pause`` bracket each region; the samples of all regions are pooled).
+    Reads only; no setting of the GPU is touched."""
 
     REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
                ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
@@ -124,6 +145,7 @@ class ClockSampler:
         self.dev = torch_device
         self.samples = []
         self.stop_evt = threading.Event()
+        self.active = threading.Event()
         self.thread = None
         self.nvml = None
         self.handle = None
@@ -145,21 +167,31 @@ class ClockSampler:
         self.thread = threading.Thread(target=self._run, daemon=True)
         self.thread.start()
 
+    def resume(self):
+        self.active.set()
+
+    def pause(self):
+        self.active.clear()
+
     def _run(self):
         nv = self.nvml
         while not self.stop_evt.is_set():
+            if not self.active.wait(0.05):
+                continue
             try:
                 mhz = nv.nvmlDeviceGetClockInfo(self.handle, nv.NVML_CLOCK_SM)
                 mask = nv.nvmlDeviceGetCurrentClocksEventReasons(self.handle)
-                self.samples.append((time.perf_counter(), mhz, mask))
+                if self.active.is_set():
+                    self.samples.append((time.perf_counter(), mhz, mask))
             except Exception:
                 pass
-            self.stop_evt.wait(0.005)
+            self.stop_evt.wait(0.001)
 
     def stop(self):
         if self.thread is None:
             return None
         self.stop_evt.set()
+        self.active.set()
         self.thread.join(timeout=5)
         if not self.samples:
             return None
@@ -346,92 +378,167 @@ class QuantCall:
     def d2h_bytes(self) -> int:
         return self.q.numel() + self.sfa.numel() * 4
 
-def run_ours(args, rank, world, local_rank):
+def make_call(workload: str, prob, dev):
+    """The call object (pinned host inputs, device outputs, library call) of a workload."""
+    if is_quant(workload):
+        return QuantCall(prob, dev)
+    if is_bf16(workload):
+        return Bf16Call(prob, dev)
+    return FFNCall(prob, dev) if prob.layout == "ffn_contiguous" else GemmCall(prob, dev)
+
+
+@dataclasses.dataclass
+class Timing:
+    """Device timing of one workload: the mean and median step time (each the
+    max over ranks) and the number of this library's kernels per step."""
+    workload: str
+    prob: object
+    ms: float
+    ms_median: float
+    launches: int
+
+
+class DeviceBench:
+    """The device side of one rank: L2 flush buffers, the launching stream, the
+    barrier that brackets every timed region and the clock sampler."""
+
+    def __init__(self, dev, world: int, local_rank: int):
+        import torch
+        self.dev, self.world, self.local_rank = dev, world, local_rank
+        self.stream = torch.cuda.current_stream(dev)
+        self.flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+        self.flush_read = torch.ones(FLUSH_BYTES // 8, dtype=torch.float32, device=dev)
+        self.sampler = ClockSampler(dev)
+
+    def flush_l2(self, i: int):
+        # write > L2 (evicts every input line), then read > L2 so the dirty lines
+        # of the write are written back now and the timed step starts from a
+        # cold, clean L2
+        self.flush.fill_(float(i))
+        self.flush_read.sum()
+
+    def barrier(self):
+        import torch
+        import torch.distributed as dist
+        if self.world > 1:
+            dist.barrier(device_ids=[self.local_rank])
+        torch.cuda.synchronize(self.dev)
+
+    def time_steps(self, step, steps: int, warmup: int):
+        """W untimed warm-up steps, then exactly K steps, each after an L2 flush
+        and timed alone with CUDA events on the launching stream; the region is
+        bracketed by a barrier and a device synchronisation on both sides.
+        Returns (mean ms, median ms), each the max over ranks."""
+        import torch
+        import moe_grouped_gemm_fp32_b200 as dg
+        for i in range(warmup):
+            self.flush_l2(i)
+            step()
+        dg.dg_get_device_status(clear=True)
+        self.barrier()
+        self.sampler.resume()
+        starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+        ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+        for i in range(steps):
+            self.flush_l2(i)                      # every step starts from HBM
+            starts[i].record(self.stream)
+            step()
+            ends[i].record(self.stream)
+        self.barrier()
+        self.sampler.pause()
+        per_step = [a.elapsed_time(b) for a, b in zip(starts, ends)]
+        status = dg.dg_get_device_status(clear=True)
+        if status:
+            raise RuntimeError(f"kernel status word {status:#x}")
+        ms, med = max_over_ranks([sum(per_step) / len(per_step), statistics.median(per_step)],
+                                 self.dev, self.world)
+        return ms, med
+
+
+def time_workload(bench: DeviceBench, workload: str, rank: int, steps: int, warmup: int,
+                  keep: bool = False):
+    """Device timing of one workload on this rank's problem; with ``keep`` also
+    the call object and its device inputs (for the end-to-end and graph timings)."""
+    prob = rank_problem(workload, rank)
+    op = make_call(workload, prob, bench.dev)
+    devt = {k: v.to(bench.dev, non_blocking=False) for k, v in op.host.items()}
+    ms, med = bench.time_steps(lambda: op.call(devt, bench.stream), steps, warmup)
+    t = Timing(workload, prob, ms, med, op.launches_per_step)
+    return (t, op, devt) if keep else t
+
+
+def launch_floor_ms(bench: DeviceBench, steps: int, warmup: int) -> float:
+    """Event-timed step of an empty kernel (torch's zero-cycle sleep kernel)
+    under the same flush and events: the timing method's own floor."""
     import torch
-    import torch.distributed as dist
-    import moe_grouped_gemm_fp32_b200 as dg
+    ms, _ = bench.time_steps(lambda: torch.cuda._sleep(0), steps, warmup)
+    return ms
+
+
+def run_ours(args, rank, world, local_rank):
+    """Times the headline workload (device-resident and end to end from pinned
+    host buffers, plus the CUDA-graph replay for masked GEMMs), then every
+    workload of ``shapes``.  Returns (headline Timing, e2e ms, h2d bytes, d2h
+    bytes, graph ms, [Timing of each shape], clocks, launch-floor ms)."""
+    import torch
     from moe_grouped_gemm_fp32_b200 import build as dg_build
 
     dg_build.build()
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    prob = rank_problem(args.workload, rank)
+    bench = DeviceBench(dev, world, local_rank)
+    bench.sampler.start()
 
-    op = (QuantCall if is_quant(args.workload) else Bf16Call if is_bf16(args.workload)
-          else FFNCall if prob.layout == "ffn_contiguous" else GemmCall)(prob, dev)
-    host = op.host
-    devt = {k: v.to(dev, non_blocking=False) for k, v in host.items()}
-    flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
-    flush_read = torch.ones(FLUSH_BYTES // 8, dtype=torch.float32, device=dev)
-
-    def flush_l2(i):
-        # write > L2 (evicts every input line), then read > L2 so the dirty lines
-        # of the write are written back now and the timed step starts from a
-        # cold, clean L2
-        flush.fill_(float(i))
-        flush_read.sum()
-    stream = torch.cuda.current_stream(dev)
-
-    def call(t):
-        op.call(t, stream)
-
-    def barrier():
-        if world > 1:
-            dist.barrier(device_ids=[local_rank])
-        torch.cuda.synchronize(dev)
-
-    sampler = ClockSampler(dev)
-    # ---- device-resident timing
-    for i in range(args.warmup):
-        flush_l2(i)
-        call(devt)
-    dg.dg_get_device_status(clear=True)
-    sampler.start()
-    barrier()
-    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    for i in range(args.steps):
-        flush_l2(i)                      # every step starts from HBM
-        starts[i].record(stream)
-        call(devt)
-        ends[i].record(stream)
-    barrier()
-    clocks = sampler.stop()
-    per_step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
-    ms = sum(per_step_ms) / len(per_step_ms)
-    ms_median = statistics.median(per_step_ms)
-    status = dg.dg_get_device_status(clear=True)
-    if status:
-        raise RuntimeError(f"kernel status word {status:#x}")
+    # ---- the headline: device-resident timing
+    head, op, devt = time_workload(bench, args.workload, rank, args.steps, args.warmup, keep=True)
+    stream = bench.stream
 
     # ---- end to end through the public API from pinned host buffers
+    host = op.host
     for _ in range(max(1, args.warmup // 2)):
         tt = {k: v.to(dev, non_blocking=True) for k, v in host.items()}
-        call(tt)
+        op.call(tt, stream)
         op.read_back()
-    barrier()
+    bench.barrier()
+    bench.sampler.resume()
     e_start = torch.cuda.Event(enable_timing=True)
     e_end = torch.cuda.Event(enable_timing=True)
     e2e_steps = max(1, min(args.steps, 50))
     e_start.record(stream)
     for _ in range(e2e_steps):
         tt = {k: v.to(dev, non_blocking=True) for k, v in host.items()}
-        call(tt)
+        op.call(tt, stream)
         op.read_back()
     e_end.record(stream)
-    barrier()
+    bench.barrier()
+    bench.sampler.pause()
     e2e_ms = e_start.elapsed_time(e_end) / e2e_steps
     h2d = sum(v.numel() * v.element_size() for v in host.values())
     d2h = op.d2h_bytes()
 
-    graph_ms = (graph_timing(op, devt, dev, stream)
-                if prob.layout == "masked" and not is_quant(args.workload) else 0.0)
+    graph_ms = 0.0
+    if head.prob.layout == "masked" and not is_quant(args.workload):
+        bench.sampler.resume()
+        graph_ms = graph_timing(op, devt, dev, stream)
+        bench.sampler.pause()
+    import moe_grouped_gemm_fp32_b200 as dg
     status = dg.dg_get_device_status(clear=True)
     if status:
         raise RuntimeError(f"kernel status word {status:#x}")
+    e2e_ms, graph_ms = max_over_ranks([e2e_ms, graph_ms], dev, world)
+    del op, devt, tt
 
-    ms, ms_median, e2e_ms, graph_ms = max_over_ranks([ms, ms_median, e2e_ms, graph_ms], dev, world)
-    return prob, ms, ms_median, e2e_ms, h2d, d2h, clocks, graph_ms, op.launches_per_step
+    # ---- the other configurations of the benchmark set, same steps and flush
+    shapes = []
+    for w in args.shape_list:
+        if w == args.workload:
+            shapes.append(head)
+            continue
+        shapes.append(time_workload(bench, w, rank, args.steps, args.warmup))
+        torch.cuda.empty_cache()
+    floor_ms = launch_floor_ms(bench, args.steps, args.warmup) if args.shape_list else 0.0
+    clocks = bench.sampler.stop()
+    return head, e2e_ms, h2d, d2h, graph_ms, shapes, clocks, floor_ms
 
 
 def graph_timing(op, devt, dev, stream, replays: int = 5) -> float:
@@ -687,17 +794,69 @@ def shape_config(prob):
     return c
 
 
+def roofline(workload: str, prob, ms: float):
+    """Roofline entry of one workload's kernel: algorithmic bytes (HBM-bound) or
+    FLOP (tensor-bound) per launch over the measured step time, against the
+    measured peak, and the ncu DRAM traffic of one launch when it is current."""
+    peaks, peak_src = measured_peaks()
+    unit = UNIT[workload]
+    if unit == "GB/s":
+        bound, peak, runit = "hbm", peaks["hbm_gbs"], "GB/s"
+        nominal = NOMINAL_PEAK["hbm"]
+        achieved = prob.bytes() / (ms * 1e-3) / 1e9
+        src = "hbm_gbs"
+    else:
+        bound, runit = "tensor", "TFLOP/s"
+        # BF16: the measured BF16 peak; FP8 dense = 2 x BF16 dense (nominal ratio)
+        peak = peaks["bf16_tflops"] * (1.0 if is_bf16(workload) else 2.0)
+        nominal = NOMINAL_PEAK["bf16" if is_bf16(workload) else "fp8"]
+        achieved = prob.flops() / (ms * 1e-3) / 1e12
+        src = "bf16_tflops" if is_bf16(workload) else "2 x bf16_tflops"
+    return {"bound": bound, "achieved": achieved, "peak": peak, "unit": runit, "frac": achieved / peak,
+            "traffic": profiled_traffic(workload), "nominal_peak": nominal,
+            "frac_of_nominal": achieved / nominal, "peak_source": f"{peak_src} ({src})"}
+
+
+def shape_entry(t: Timing, world: int):
+    unit = UNIT[t.workload]
+    e = {"value": metric_value(t.prob, unit, t.ms, world), "unit": unit, "ms_per_step": t.ms,
+         "ms_median": t.ms_median, "launches_per_step": t.launches,
+         "roofline": roofline(t.workload, t.prob, t.ms), "config": shape_config(t.prob)}
+    pages = PAGES_NUMBER.get(t.workload)
+    if pages and pages[1] == unit:
+        e["vs_pages"] = e["value"] / pages[0]
+    return e
+
+
+def parse_shapes(arg: str, workload: str):
+    if arg == "none":
+        return []
+    if arg == "auto":
+        return list(SHAPES) if workload == DEFAULT_WORKLOAD else []
+    names = [w for w in arg.split(",") if w]
+    for w in names:
+        if w not in UNIT:
+            raise SystemExit(f"unknown workload {w!r}")
+    return names
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=100)
-    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--shapes", default="auto",
+                    help="workloads timed after the headline under 'shapes': auto (the benchmark "
+                         "set when the headline is the default workload), none, or a comma list")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.workload not in UNIT:
+        ap.error(f"unknown workload {args.workload!r}")
+    args.shape_list = parse_shapes(args.shapes, args.workload)
 
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -713,26 +872,22 @@ def main():
         dist.init_process_group("nccl", timeout=timedelta(seconds=300),
                                 device_id=torch.device("cuda", local_rank))
     try:
-        prob, ms, ms_median, e2e_ms, h2d, d2h, clocks, graph_ms, launches = run_ours(args, rank, world, local_rank)
+        head, e2e_ms, h2d, d2h, graph_ms, shapes, clocks, floor_ms = run_ours(args, rank, world, local_rank)
     finally:
         if world > 1:
             dist.destroy_process_group()
     if rank != 0:
         return 0
-    unit = UNIT[args.workload]
+    prob, ms, unit = head.prob, head.ms, UNIT[args.workload]
     value = metric_value(prob, unit, ms, world)
-    peaks, peak_src = measured_peaks()
-    if unit == "GB/s":
-        bound, peak, runit = "hbm", peaks["hbm_gbs"], "GB/s"
-        nominal = NOMINAL_PEAK["hbm"]
-        achieved = prob.bytes() / (ms * 1e-3) / 1e9
-    else:
-        bound, runit = "tensor", "TFLOP/s"
-        # BF16: the measured BF16 peak; FP8 dense = 2 x BF16 dense (nominal ratio)
-        peak = peaks["bf16_tflops"] * (1.0 if is_bf16(args.workload) else 2.0)
-        nominal = NOMINAL_PEAK["bf16" if is_bf16(args.workload) else "fp8"]
-        achieved = prob.flops() / (ms * 1e-3) / 1e12
     pages = PAGES_NUMBER.get(args.workload)
+    measurement = {"l2": "flushed before every step (512 MB write, then 256 MB read)",
+                   "gbps": prob.bytes() / (ms * 1e-3) / 1e9, "ms_median_step": head.ms_median}
+    if not is_quant(args.workload):
+        measurement["tflops"] = prob.flops() / (ms * 1e-3) / 1e12
+    if floor_ms > 0:
+        measurement["launch_floor_ms"] = floor_ms
+        measurement["launch_floor"] = "an empty kernel timed the same way (flush, events around one launch)"
     line = {
         "metric": METRIC, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
@@ -741,23 +896,20 @@ def main():
                   else "bf16 (f32 accumulate, bf16 out)" if is_bf16(args.workload)
                   else "e4m3 (f32 accumulate, bf16 out)"),
         "data": "synthetic",
-        "config": {"workload": args.workload, **shape_config(prob),
-                   "l2": "flushed before every step (512 MB write, then 256 MB read)",
-                   **({} if is_quant(args.workload) else {"tflops": prob.flops() / (ms * 1e-3) / 1e12}),
-                   "gbps": prob.bytes() / (ms * 1e-3) / 1e9, "ms_median_step": ms_median},
-        "roofline": {"bound": bound, "achieved": achieved, "peak": peak, "unit": runit,
-                     "frac": achieved / peak, "traffic": profiled_traffic(args.workload),
-                     "nominal_peak": nominal, "frac_of_nominal": achieved / nominal,
-                     "peak_source": f"{peak_src} ({'hbm_gbs' if bound == 'hbm' else 'bf16_tflops' if is_bf16(args.workload) else '2 x bf16_tflops'})"},
+        "config": {"workload": args.workload, **shape_config(prob)},
+        "roofline": roofline(args.workload, prob, ms),
         "e2e": {"value": metric_value(prob, unit, e2e_ms, world), "unit": unit,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": args.steps * launches,
+        "gpu_launches": args.steps * head.launches,
         "clocks": clocks,
+        "measurement": measurement,
     }
     if graph_ms > 0:
         line["graph"] = {"value": metric_value(prob, unit, graph_ms, world), "unit": unit,
                          "ms_per_call": graph_ms, "calls_per_graph": GRAPH_CALLS,
                          "l2": "not flushed between calls (B alone exceeds L2)"}
+    if shapes:
+        line["shapes"] = {t.workload: shape_entry(t, world) for t in shapes}
     if not args.no_cpu_baseline and world == 1:
         cb = cpu_baseline(prob, unit)
         cb.pop("seconds_per_step", None)

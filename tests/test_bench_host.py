@@ -126,12 +126,14 @@ def test_reference_arm_for_the_next_rows(workload):
 def test_our_json_line_carries_every_contract_key(monkeypatch, capsys, workload, launches, graph):
     """The line of our arm, assembled from a stubbed device run: every key the
     bench contract names is present, with the roofline fraction, the launch
-    count and (masked GEMMs only) the CUDA-graph figure consistent."""
+    count and (masked GEMMs only) the CUDA-graph figure consistent; the
+    workload config holds no measurement."""
     prob = bench.rank_problem(workload, 0)
-    clocks = {"sm_mhz": 1965, "sm_max_mhz": 1965, "reasons": []}
+    clocks = {"sm_mhz": 1965, "sm_max_mhz": 1965, "reasons": [], "samples": 40}
+    head = bench.Timing(workload, prob, 0.5, 0.49, launches)
     monkeypatch.setattr(bench, "run_ours",
-                        lambda args, rank, world, lr: (prob, 0.5, 0.49, 0.8, 100, 20, clocks,
-                                                       0.51 if graph else 0.0, launches))
+                        lambda args, rank, world, lr: (head, 0.8, 100, 20, 0.51 if graph else 0.0, [],
+                                                       clocks, 0.0))
     monkeypatch.setattr(sys, "argv", ["bench.py", "--workload", workload, "--steps", "7", "--warmup", "3",
                                       "--no-cpu-baseline"])
     assert bench.main() == 0
@@ -140,9 +142,11 @@ def test_our_json_line_carries_every_contract_key(monkeypatch, capsys, workload,
     line = json.loads(out[0])
     for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
                 "scaling", "vs_baseline", "dtype", "data", "config", "roofline", "e2e", "gpu_launches",
-                "clocks"):
+                "clocks", "measurement"):
         assert key in line, key
-    assert line["config"]["workload"] == workload and line["scaling"] == "weak"
+    assert line["config"] == {"workload": workload, **bench.shape_config(prob)}
+    assert not set(line["config"]) & {"l2", "tflops", "gbps", "ms_median_step"}
+    assert line["scaling"] == "weak"
     roof = line["roofline"]
     for key in ("bound", "achieved", "peak", "unit", "frac", "traffic"):
         assert key in roof, key
@@ -152,3 +156,61 @@ def test_our_json_line_carries_every_contract_key(monkeypatch, capsys, workload,
     assert line["gpu_launches"] == 7 * launches
     assert ("graph" in line) == graph
     assert line["clocks"] == clocks
+    assert "shapes" not in line
+
+
+def test_default_run_is_the_contiguous_prefill_with_every_shape(monkeypatch, capsys):
+    """With no flags the headline is the largest configuration (the contiguous
+    MoE prefill) and ``shapes`` carries every configuration of the benchmark set,
+    each with its own roofline entry; the reference arm names the same config."""
+    assert bench.DEFAULT_WORKLOAD == "contiguous_g4"
+    assert set(bench.SHAPES) == {"dense_tiny", "dense_decode_m64", "dense_decode_m128", "dense_large",
+                                 "contiguous_g4", "masked_g16"}
+    tiny = bench.rank_problem("dense_tiny", 0)
+    probs = {w: tiny for w in bench.SHAPES}     # stand-in problems: the accounting is per workload
+
+    def fake(args, rank, world, lr):
+        assert args.shape_list == list(bench.SHAPES)
+        shapes = [bench.Timing(w, probs[w], 0.01 * (i + 1), 0.01, 1) for i, w in enumerate(args.shape_list)]
+        head = shapes[args.shape_list.index("contiguous_g4")]
+        return head, 0.9, 10, 10, 0.0, shapes, {"sm_mhz": 1965, "sm_max_mhz": 1965, "reasons": []}, 0.006
+    monkeypatch.setattr(bench, "run_ours", fake)
+    monkeypatch.setattr(sys, "argv", ["bench.py", "--steps", "5", "--warmup", "3", "--no-cpu-baseline"])
+    assert bench.main() == 0
+    line = json.loads(capsys.readouterr().out.strip())
+    assert line["config"]["workload"] == "contiguous_g4"
+    assert set(line["shapes"]) == set(bench.SHAPES)
+    for w, e in line["shapes"].items():
+        assert e["unit"] == bench.UNIT[w]
+        assert set(e["roofline"]) >= {"achieved", "peak", "frac", "traffic"}
+        assert abs(e["roofline"]["frac"] - e["roofline"]["achieved"] / e["roofline"]["peak"]) < 1e-12
+    assert line["shapes"]["contiguous_g4"]["ms_per_step"] == line["ms_per_step"]
+    assert "vs_pages" in line["shapes"]["dense_decode_m64"]
+    assert line["vs_baseline"] is None            # no page row states all of M, N and K of this workload
+    assert line["measurement"]["launch_floor_ms"] == 0.006
+
+
+def test_shape_selection():
+    assert bench.parse_shapes("auto", "contiguous_g4") == list(bench.SHAPES)
+    assert bench.parse_shapes("auto", "dense_large") == []
+    assert bench.parse_shapes("none", "contiguous_g4") == []
+    assert bench.parse_shapes("dense_tiny,masked_g16", "dense_large") == ["dense_tiny", "masked_g16"]
+    with pytest.raises(SystemExit):
+        bench.parse_shapes("dense_tiny,nope", "dense_large")
+
+
+def test_traffic_comes_from_the_capture_file_only_while_the_sources_match(monkeypatch, tmp_path):
+    """roofline.traffic is read from a machine-readable capture file keyed by
+    kernel and workload, and only while the kernel sources hash to the value
+    recorded with the capture."""
+    f = tmp_path / "traffic.json"
+    h = bench.kernel_source_hash("fp8_gemm_kernel")
+    f.write_text(json.dumps({"captures": {
+        "fp8_gemm_kernel/dense_large": {"kernel_source_hash": h, "dram_bytes_per_launch": 123.0},
+        "fp8_gemm_kernel/masked_g16": {"kernel_source_hash": "0" * 16, "dram_bytes_per_launch": 5.0}}}))
+    monkeypatch.setattr(bench, "TRAFFIC_FILE", str(f))
+    assert bench.profiled_traffic("dense_large") == 123.0
+    assert bench.profiled_traffic("masked_g16") is None           # stale capture
+    assert bench.profiled_traffic("contiguous_g4") is None        # no capture
+    monkeypatch.setattr(bench, "TRAFFIC_FILE", str(tmp_path / "missing.json"))
+    assert bench.profiled_traffic("dense_large") is None
