@@ -907,44 +907,28 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
                     if (++buf == kAccBufs) { buf = 0; tphase ^= 1u; }
                     continue;
                 } else if constexpr (!kSwap) {
-                    // Normal mode: this warpgroup's kHalf columns in rounds of up to 32,
-                    // loaded two rounds ahead into a pair of 32-register buffers.  Rounds
-                    // 0 and 1 load before the first wait; round r + 2 loads into the
-                    // buffer round r has just consumed; a wait before every even round
-                    // from 2 on covers the two loads issued since the previous wait.  The
-                    // partial buffer is released at the wait that covers the last round,
-                    // i.e. after about half of the FMAs instead of before the last round's,
-                    // so the MMA can reuse it sooner.  Every 8-column group lies inside
-                    // one 128-row weight block (scale sblk[]).
+                    // Normal mode: this warpgroup's kHalf columns in rounds of up to 32;
+                    // each round loads its columns before one wait (the compiler may
+                    // hoist the next round's load above this round's FMAs).  Every
+                    // 8-column group lies inside one 128-row weight block (scale sblk[]).
                     constexpr int kRounds = (kHalf + 31) / 32;
                     float sblk[kNumSB];
 #pragma unroll
                     for (int i = 0; i < kNumSB; ++i) sblk[i] = sa_row * sbv[i];
-                    // this warpgroup's tile columns for round r (SwiGLU: two gate
-                    // rounds, then the two matching up rounds)
-                    auto rcol_of = [&](int r) {
-                        return kSwiGLU ? (r < 2 ? 64 * half + 32 * r : 128 + 64 * half + 32 * (r - 2))
-                                       : half * kHalf + r * 32;
-                    };
-                    auto ncol_of = [&](int r) { return (r + 1) * 32 <= kHalf ? 32 : kHalf - r * 32; };  // 32 or 16
-                    auto load_round = [&](int r, float *v) {
-                        const uint32_t ta = taddr + static_cast<uint32_t>(rcol_of(r));
-                        if (ncol_of(r) == 32) ptx::tmem_ld32p(ta, v);
-                        else ptx::tmem_ld16p(ta, v);
-                    };
-                    float vbuf[2][32];
-                    load_round(0, vbuf[0]);
-                    if (kRounds > 1) load_round(1, vbuf[1]);
-                    ptx::tmem_wait_ld();
-                    if (kRounds <= 2) release_tmem(tempty_target);
 #pragma unroll
                     for (int r = 0; r < kRounds; ++r) {
-                        if (r >= 2 && r % 2 == 0) {
-                            ptx::tmem_wait_ld();              // rounds r and r + 1 have landed
-                            if (r + 2 >= kRounds) release_tmem(tempty_target);
-                        }
-                        float *v = vbuf[r & 1];
-                        const int ncol = ncol_of(r), rcol = rcol_of(r);
+                        constexpr int kFull = 32;
+                        const int ncol = (r + 1) * 32 <= kHalf ? kFull : kHalf - r * 32;   // 32 or 16
+                        float v[32];
+                        // this warpgroup's tile columns for round r (SwiGLU: two gate
+                        // rounds, then the two matching up rounds)
+                        const int rcol = kSwiGLU ? (r < 2 ? 64 * half + 32 * r : 128 + 64 * half + 32 * (r - 2))
+                                                 : half * kHalf + r * 32;
+                        const uint32_t ta = taddr + static_cast<uint32_t>(rcol);
+                        if (ncol == 32) ptx::tmem_ld32p(ta, v);
+                        else ptx::tmem_ld16p(ta, v);
+                        ptx::tmem_wait_ld();
+                        if (r == kRounds - 1) release_tmem(tempty_target);
 #pragma unroll
                         for (int q = 0; q < 4; ++q) {
                             if (q * 8 < ncol) {
@@ -959,7 +943,6 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
                                     ptx::ffma2(a[i], a[i + 1], sc, v[q * 8 + i], v[q * 8 + i + 1]);
                             }
                         }
-                        if (r + 2 < kRounds) load_round(r + 2, vbuf[r & 1]);   // refill the buffer just used
                     }
                     if (++stage == kStages) { stage = 0; phase ^= 1u; }
                     if (++buf == kAccBufs) { buf = 0; tphase ^= 1u; }
