@@ -194,6 +194,45 @@ DG_API dg_status_t dg_m_grouped_fp8_ffn_contiguous(const uint8_t *a, const float
                                                    int I, int G, void *stream);
 
 /*
+ * The fused expert FFN above for callers that cannot allocate device memory.
+ * The pages have no counterpart: this entry point exists for users of this
+ * library, not for the method.  Some callers cannot call cudaMalloc at the
+ * point where they run the FFN: a plugin that runs inside another runtime's
+ * execution step, where the host runtime owns all device memory and forbids
+ * allocation; a serving loop that freezes its memory after warm-up so that
+ * it can never fail or stall on an allocation mid-request; a plain C program
+ * with no device allocator of its own.  Such a caller still passes its inputs
+ * and its output, but not the intermediate buffers q_mid and s_mid: the call
+ * keeps them in one file-scope device array of DG_NOALLOC_SCRATCH_BYTES bytes,
+ * which every GPU that loads this library holds until the process exits.
+ *   Arguments: as for dg_m_grouped_fp8_ffn_contiguous, without q_mid, s_mid
+ *   and ld_mid.
+ *   Size limit: the intermediate takes M_total * I bytes of E4M3 codes
+ *   (rounded up to 256) plus (I / 128) * ld * 4 bytes of scales, with ld =
+ *   M_total rounded up to a multiple of 4 (at least 4).  A call that needs
+ *   more than DG_NOALLOC_SCRATCH_BYTES returns DG_ERR_UNSUPPORTED_SHAPE before
+ *   enqueueing anything.
+ *   Set-up: the first call on a device looks up the array's device address
+ *   (cudaGetSymbolAddress, with that device current) and caches it; make that
+ *   first call before any stream capture.
+ *   Sharing: every call on a device uses the same array, which keeps the last
+ *   call's contents.  Nothing in it has to start at zero: the second GEMM reads
+ *   only intermediate rows that the first GEMM wrote in the same call.  Calls
+ *   that overlap on the GPU (on different streams, or from different threads
+ *   without ordering) race on the array and give wrong results; the caller
+ *   must order them.
+ *   The call allocates nothing: no cudaMalloc, no cudaFree, no allocating
+ *   library routine.
+ */
+#define DG_NOALLOC_SCRATCH_BYTES (16u * 1024u * 1024u)
+DG_API dg_status_t dg_m_grouped_fp8_ffn_contiguous_noalloc(const uint8_t *a, const float *sfa,
+                                                           int ld_sfa, const uint8_t *w1,
+                                                           const float *sfb1, const uint8_t *w2,
+                                                           const float *sfb2, void *y,
+                                                           const int32_t *m_indices, int M_total,
+                                                           int H, int I, int G, void *stream);
+
+/*
  * BF16 GEMMs (page 3 "核心功能": FP8, FP4 and BF16 GEMM operations, in the same
  * dense and m-grouped layouts):
  *   D[m,n] = sum_k A[m,k] * B[n,k]    accumulated in FP32, stored as BF16 (RNE)

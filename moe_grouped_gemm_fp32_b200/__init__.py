@@ -63,6 +63,7 @@ def lib() -> ctypes.CDLL:
     L.dg_k_grouped_fp8_gemm_nt_contiguous.argtypes = [P, P, I, P, P, P, P, I, I, I, I, P]
     L.dg_m_grouped_fp8_gemm_swiglu_quant_contiguous.argtypes = [P, P, I, P, P, P, P, I, P, I, I, I, I, P]
     L.dg_m_grouped_fp8_ffn_contiguous.argtypes = [P, P, I, P, P, P, P, P, P, I, P, P, I, I, I, I, P]
+    L.dg_m_grouped_fp8_ffn_contiguous_noalloc.argtypes = [P, P, I, P, P, P, P, P, P, I, I, I, I, P]
     L.dg_bf16_gemm_nt.argtypes = [P, P, P, I, I, I, P]
     L.dg_m_grouped_bf16_gemm_nt_contiguous.argtypes = [P, P, P, P, I, I, I, I, P]
     L.dg_m_grouped_bf16_gemm_nt_masked.argtypes = [P, P, P, P, I, I, I, I, P]
@@ -301,6 +302,35 @@ def dg_m_grouped_fp8_ffn_contiguous(a, sfa, w1, sfb1, w2, sfb2, q_mid, s_mid, y,
           (a, sfa, w1, sfb1, w2, sfb2, q_mid, s_mid, y, m_indices), stream,
           ptrs[0], ptrs[1], sfa.shape[-1], ptrs[2], ptrs[3], ptrs[4], ptrs[5], ptrs[6], ptrs[7],
           s_mid.shape[-1], ptrs[8], ptrs[9], M_total, H, I, G)
+    return y
+
+
+def dg_m_grouped_fp8_ffn_contiguous_noalloc(a, sfa, w1, sfb1, w2, sfb2, y, m_indices, stream=None):
+    """The fused expert FFN for callers that cannot allocate device memory: as
+    dg_m_grouped_fp8_ffn_contiguous, but the intermediate codes and scales live
+    in the library's own fixed device array (DG_NOALLOC_SCRATCH_BYTES, 16 MiB),
+    so nothing is allocated, here or in the C call.  Calls that overlap on the
+    GPU share that array and race; order them."""
+    import torch
+    ptrs = (_req(a, torch.uint8, "a", 2), _req(sfa, torch.float32, "sfa", 2),
+            _req(w1, torch.uint8, "w1", 3), _req(sfb1, torch.float32, "sfb1", 3),
+            _req(w2, torch.uint8, "w2", 3), _req(sfb2, torch.float32, "sfb2", 3),
+            _req(y, torch.bfloat16, "y", 2), _req(m_indices, torch.int32, "m_indices", 1))
+    M_total, H = a.shape
+    G, I2, _ = w1.shape
+    I = I2 // 2
+    HB, IB = _blocks(H), _blocks(I)
+    _shape(sfa, (HB, None), "sfa")
+    _shape(w1, (G, 2 * I, H), "w1")
+    _shape(sfb1, (G, _ceil_blocks(2 * I), HB), "sfb1")
+    _shape(w2, (G, H, I), "w2")
+    _shape(sfb2, (G, _ceil_blocks(H), IB), "sfb2")
+    _shape(y, (M_total, H), "y")
+    _shape(m_indices, (M_total,), "m_indices")
+    _call("dg_m_grouped_fp8_ffn_contiguous_noalloc", lib().dg_m_grouped_fp8_ffn_contiguous_noalloc,
+          (a, sfa, w1, sfb1, w2, sfb2, y, m_indices), stream,
+          ptrs[0], ptrs[1], sfa.shape[-1], ptrs[2], ptrs[3], ptrs[4], ptrs[5], ptrs[6], ptrs[7],
+          M_total, H, I, G)
     return y
 
 # --------------------------------------------------------------------------- BF16 GEMMs

@@ -600,6 +600,63 @@ dg_status_t dg_m_grouped_fp8_ffn_contiguous(const uint8_t *a, const float *sfa, 
                                                stream);
 }
 
+}  // extern "C"
+
+// ------------------------------------------------------------ no-allocation FFN
+namespace {
+// The intermediate of dg_m_grouped_fp8_ffn_contiguous_noalloc (E4M3 codes, then
+// their scales) lives in this file-scope device array, for callers that cannot
+// allocate device memory.  Every GPU that loads the library holds it until exit.
+__device__ __align__(256) unsigned char g_noalloc_scratch[DG_NOALLOC_SCRATCH_BYTES];
+
+// The array's device address on each device.  In host code the name
+// g_noalloc_scratch is only a host-side stand-in, not a device address (a kernel
+// given it would fault, or silently use host memory where the GPU can reach it),
+// so the address is looked up once per device, with that device current.
+std::atomic<void *> g_noalloc_addr[kMaxDevices];
+
+dg_status_t noalloc_scratch(void **out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (dev < 0 || dev >= kMaxDevices) return DG_ERR_UNSUPPORTED_DEVICE;
+    void *p = g_noalloc_addr[dev].load(std::memory_order_acquire);
+    if (!p) {
+        if ((e = cudaGetSymbolAddress(&p, g_noalloc_scratch)) != cudaSuccess)
+            return cuda_fail(e, "cudaGetSymbolAddress(no-allocation scratch)");
+        g_noalloc_addr[dev].store(p, std::memory_order_release);
+    }
+    *out = p;
+    return DG_SUCCESS;
+}
+}  // namespace
+
+extern "C" {
+
+dg_status_t dg_m_grouped_fp8_ffn_contiguous_noalloc(const uint8_t *a, const float *sfa, int ld_sfa,
+                                                    const uint8_t *w1, const float *sfb1,
+                                                    const uint8_t *w2, const float *sfb2, void *y,
+                                                    const int32_t *m_indices, int M_total, int H,
+                                                    int I, int G, void *stream) {
+    if (M_total < 0) return DG_ERR_INVALID_VALUE;
+    if (I <= 0 || I % 128 != 0) return DG_ERR_UNSUPPORTED_SHAPE;
+    // intermediate: codes [M_total][I], then scales [I/128][ld_mid] at a 256-byte offset
+    const long long ld_mid = M_total < 4 ? 4 : (static_cast<long long>(M_total) + 3) / 4 * 4;
+    const long long s_offset = (static_cast<long long>(M_total) * I + 255) / 256 * 256;
+    const long long need = s_offset + static_cast<long long>(I / 128) * ld_mid * 4;
+    if (need > static_cast<long long>(DG_NOALLOC_SCRATCH_BYTES)) return DG_ERR_UNSUPPORTED_SHAPE;
+    const DeviceInfo *info = nullptr;
+    dg_status_t st = device_info(&info);
+    if (st != DG_SUCCESS) return st;
+    void *scratch = nullptr;
+    if ((st = noalloc_scratch(&scratch)) != DG_SUCCESS) return st;
+    uint8_t *q_mid = static_cast<uint8_t *>(scratch);
+    float *s_mid = reinterpret_cast<float *>(static_cast<unsigned char *>(scratch) + s_offset);
+    return dg_m_grouped_fp8_ffn_contiguous(a, sfa, ld_sfa, w1, sfb1, w2, sfb2, q_mid, s_mid,
+                                           static_cast<int>(ld_mid), y, m_indices, M_total, H, I, G,
+                                           stream);
+}
+
 int dg_get_m_alignment_for_contiguous_layout(void) { return 128; }
 
 size_t dg_get_tma_aligned_size(size_t n, size_t elem_bytes) {
