@@ -826,6 +826,28 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
     auto col_of = [&](int c) {                       // first tile column of local chunk c
         return kSwap ? (2 * c + half) * kChunk : half * kHalf + c * kChunk;
     };
+    // Normal mode, tiles wider than 192: the tile column of this warpgroup's
+    // 32-column round r (the last round may hold 16).  Tiles start on a multiple
+    // of 32 (224-wide) or of 256, so every 128-row weight-block boundary inside a
+    // tile lies on a multiple of 32 relative to it.  256-wide tiles give each
+    // warpgroup one contiguous half, whose rounds start on multiples of 32; the
+    // SwiGLU epilogue's warpgroup takes two gate rounds, then the two matching up
+    // rounds.  224-wide tiles interleave the six full rounds between the
+    // warpgroups (round r of warpgroup h is tile columns 32 (2r + h) ..) and split
+    // the last 32 columns 16/16 (no boundary at 208).  Either way no round
+    // straddles a weight block.
+    constexpr bool kInterleave = !kSwap && kHalf > 96 && kHalf % 32 != 0;
+    auto round_col = [&](int r) -> int {
+        if constexpr (kSwiGLU) return r < 2 ? 64 * half + 32 * r : 128 + 64 * half + 32 * (r - 2);
+        if constexpr (kInterleave) return r < kHalf / 32 ? 32 * (2 * r + half) : 2 * (kHalf / 32) * 32 + 16 * half;
+        return half * kHalf + r * 32;
+    };
+    // tile column of this thread's accumulator j (normal mode)
+    auto out_col = [&](int j) -> int {
+        if constexpr (kInterleave) return round_col(j / 32) + j % 32;
+        return half * kHalf + j;
+    };
+    static_assert(!kInterleave || kBN == 224, "interleaved rounds are laid out for 224-wide tiles");
     // the partial buffers are released on the MMA CTA's barrier (remote for a pair's second CTA)
     const bool remote_release = kPair && !mma_cta;
     const uint32_t tempty_target0 = remote_release ? leader_addr(tempty_bar(0)) : tempty_bar(0);
@@ -907,10 +929,10 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
                     if (++buf == kAccBufs) { buf = 0; tphase ^= 1u; }
                     continue;
                 } else if constexpr (!kSwap) {
-                    // Normal mode: this warpgroup's kHalf columns in rounds of up to 32;
-                    // each round loads its columns before one wait (the compiler may
-                    // hoist the next round's load above this round's FMAs).  Every
-                    // 8-column group lies inside one 128-row weight block (scale sblk[]).
+                    // Normal mode: this warpgroup's kHalf columns in rounds of up to 32
+                    // (round_col() gives their place in the tile); each round loads its
+                    // columns before one wait.  No round straddles a 128-row weight
+                    // block, so each round takes one scale, chosen once per round.
                     constexpr int kRounds = (kHalf + 31) / 32;
                     float sblk[kNumSB];
 #pragma unroll
@@ -920,29 +942,20 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
                         constexpr int kFull = 32;
                         const int ncol = (r + 1) * 32 <= kHalf ? kFull : kHalf - r * 32;   // 32 or 16
                         float v[32];
-                        // this warpgroup's tile columns for round r (SwiGLU: two gate
-                        // rounds, then the two matching up rounds)
-                        const int rcol = kSwiGLU ? (r < 2 ? 64 * half + 32 * r : 128 + 64 * half + 32 * (r - 2))
-                                                 : half * kHalf + r * 32;
+                        const int rcol = round_col(r);
                         const uint32_t ta = taddr + static_cast<uint32_t>(rcol);
                         if (ncol == 32) ptx::tmem_ld32p(ta, v);
                         else ptx::tmem_ld16p(ta, v);
                         ptx::tmem_wait_ld();
                         if (r == kRounds - 1) release_tmem(tempty_target);
+                        const int blk = (tl.n0 + rcol) / 128 - wblk0;
+                        float sc = sblk[0];
 #pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            if (q * 8 < ncol) {
-                                const int col = rcol + q * 8;
-                                const int blk = (tl.n0 + col) / 128 - wblk0;
-                                float sc = sblk[0];
+                        for (int i = 1; i < kNumSB; ++i) sc = blk == i ? sblk[i] : sc;
+                        float *a = acc + r * 32;
 #pragma unroll
-                                for (int i = 1; i < kNumSB; ++i) sc = blk == i ? sblk[i] : sc;
-                                float *a = acc + r * 32 + q * 8;
-#pragma unroll
-                                for (int i = 0; i < 8; i += 2)
-                                    ptx::ffma2(a[i], a[i + 1], sc, v[q * 8 + i], v[q * 8 + i + 1]);
-                            }
-                        }
+                        for (int i = 0; i < 32; i += 2)
+                            if (i < ncol) ptx::ffma2(a[i], a[i + 1], sc, v[i], v[i + 1]);
                     }
                     if (++stage == kStages) { stage = 0; phase ^= 1u; }
                     if (++buf == kAccBufs) { buf = 0; tphase ^= 1u; }
@@ -1074,7 +1087,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
                             make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
                     ptx::fence_proxy_async_smem();
                     __syncwarp();
-                    const int col0 = tl.n0 + half * kHalf + c * 32;
+                    const int col0 = tl.n0 + out_col(c * 32);
                     if (lane == 0 && rows_in && col0 < p.N) {
                         ptx::tma_store_2d(&tm_d, box_s, col0, drow0);
                         ptx::bulk_commit();
@@ -1088,7 +1101,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
                         __nv_bfloat16 *drow = p.d + (row_base + my_tok) * static_cast<size_t>(p.N);
 #pragma unroll
                         for (int j = kFull * 32; j < kHalf; j += 8) {
-                            const int col = tl.n0 + half * kHalf + j;
+                            const int col = tl.n0 + out_col(j);
                             if (col < p.N) {
                                 uint4 pk;
                                 __nv_bfloat162 h0 = __floats2bfloat162_rn(acc[j + 0], acc[j + 1]);
@@ -1109,7 +1122,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
                     __nv_bfloat16 *drow = p.d + (row_base + my_tok) * static_cast<size_t>(p.N);
 #pragma unroll
                     for (int j = 0; j < kHalf; j += 8) {
-                        const int col = tl.n0 + half * kHalf + j;
+                        const int col = tl.n0 + out_col(j);
                         if (col < p.N) {
                             uint4 pk;
                             __nv_bfloat162 h0 = __floats2bfloat162_rn(acc[j + 0], acc[j + 1]);
