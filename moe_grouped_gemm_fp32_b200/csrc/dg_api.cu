@@ -380,8 +380,8 @@ dg_status_t dg_fp8_gemm_nt(const uint8_t *a, const float *sfa, int ld_sfa, const
         if ((st = make_map(&mb, b, K, N, 1, 128)) != DG_SUCCESS) return st;
         return launch<128, false, 6, dg::kDense>(ma, mb, md, p, grid, 1, 1, s);
     }
-    // CTA pairs: 256 x bn tiles with tcgen05.mma.cta_group::2 (DG_PAIR_N
-    // overrides bn for tuning sweeps)
+    // CTA pairs: 256 x bn tiles with tcgen05.mma.cta_group::2 (DG_PAIR_N =
+    // 128 / 160 / 224 / 256 overrides bn for tuning sweeps)
     static const int forced_bn = [] {
         const char *e = std::getenv("DG_PAIR_N");
         return e ? std::atoi(e) : 0;
@@ -391,14 +391,16 @@ dg_status_t dg_fp8_gemm_nt(const uint8_t *a, const float *sfa, int ld_sfa, const
     const int pm256 = max_active_clusters<256, false, 6, dg::kDense, 2>(2);
     int bn = pair_efficiency(row_pairs, N, 224, pm224) > pair_efficiency(row_pairs, N, 256, pm256) + 1e-9
                  ? 224 : 256;
-    if (forced_bn == 160 || forced_bn == 224 || forced_bn == 256) bn = forced_bn;
-    const int pairs_max = bn == 160   ? max_active_clusters<160, false, 7, dg::kDense, 2>(2)
+    if (forced_bn == 128 || forced_bn == 160 || forced_bn == 224 || forced_bn == 256) bn = forced_bn;
+    const int pairs_max = bn == 128   ? max_active_clusters<128, false, 8, dg::kDense, 2>(2)
+                          : bn == 160 ? max_active_clusters<160, false, 7, dg::kDense, 2>(2)
                           : bn == 224 ? pm224 : pm256;
     if (pairs_max <= 0) return cuda_fail(cudaErrorInvalidConfiguration, "no resident CTA pair");
     const int tiles = ((M + 255) / 256) * ((N + bn - 1) / bn);
     const int pairs = tiles < pairs_max ? tiles : pairs_max;
     if ((st = make_map(&ma, a, K, M, 1, 128)) != DG_SUCCESS) return st;
     if ((st = make_map(&mb, b, K, N, 1, bn / 2)) != DG_SUCCESS) return st;
+    if (bn == 128) return launch<128, false, 8, dg::kDense, 2>(ma, mb, md, p, 2 * pairs, 1, 2, s);
     if (bn == 160) return launch<160, false, 7, dg::kDense, 2>(ma, mb, md, p, 2 * pairs, 1, 2, s);
     if (bn == 224) return launch<224, false, 6, dg::kDense, 2>(ma, mb, md, p, 2 * pairs, 1, 2, s);
     return launch<256, false, 6, dg::kDense, 2>(ma, mb, md, p, 2 * pairs, 1, 2, s);

@@ -914,17 +914,21 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
                     float sblk[kNumSB];
 #pragma unroll
                     for (int i = 0; i < kNumSB; ++i) sblk[i] = sa_row * sbv[i];
+                    // one scale per 16 columns: tiles start on multiples of 32 and the
+                    // warpgroup halves on multiples of 16, so no 16-column group
+                    // straddles a 128-row weight block
 #pragma unroll
-                    for (int q = 0; q < kHalf / 8; ++q) {
-                        const int col = half * kHalf + q * 8;
+                    for (int q = 0; q < kHalf / 16; ++q) {
+                        const int col = half * kHalf + q * 16;
                         const int blk = (tl.n0 + col) / 128 - wblk0;
                         float sc = sblk[0];
 #pragma unroll
                         for (int i = 1; i < kNumSB; ++i) sc = blk == i ? sblk[i] : sc;
 #pragma unroll
-                        for (int i = 0; i < 8; i += 2)
-                            ptx::ffma2(acc[q * 8 + i], acc[q * 8 + i + 1], sc, v[q * 8 + i], v[q * 8 + i + 1]);
+                        for (int i = 0; i < 16; i += 2)
+                            ptx::ffma2(acc[q * 16 + i], acc[q * 16 + i + 1], sc, v[q * 16 + i], v[q * 16 + i + 1]);
                     }
+                    static_assert(kHalf % 16 == 0, "16-column scale groups");
                     if (++stage == kStages) { stage = 0; phase ^= 1u; }
                     if (++buf == kAccBufs) { buf = 0; tphase ^= 1u; }
                     continue;

@@ -104,3 +104,21 @@ def test_ffn_full_width_all_rows():
     assert len(rows) >= 512
     ref = oracle.ffn_rows(prob, rows)
     compare(y.double().cpu().numpy()[rows], ref["y"], np.ones(ref["y"].shape, bool))
+
+
+@pytest.mark.parametrize("bn", [128, 160, 224, 256])
+def test_dense_pair_tile_widths(bn):
+    """Every CTA-pair tile width the dense path can take (DG_PAIR_N forces it,
+    in a child process): 1280 x 2112 (a weight tail) x 2048, whole output."""
+    import os, subprocess, sys
+    code = ("import sys; sys.path[:0] = [%r, %r]\n"
+            "import workloads as W, oracle\n"
+            "from gpu_util import DeviceProblem, compare, to_f64, valid_mask\n"
+            "p = W.make_dense(1280, 2112, 2048, seed=307, outliers=True)\n"
+            "dp = DeviceProblem(p); dp.fill_sentinel(); d = to_f64(dp.run())\n"
+            "compare(d, oracle.solve(p), valid_mask(p)); print('OK')\n"
+            % (os.path.dirname(os.path.dirname(__file__)), os.path.dirname(__file__)))
+    env = dict(os.environ, DG_PAIR_N=str(bn), DG_VERBOSE="1")
+    r = subprocess.run([sys.executable, "-c", code], env=env, capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0 and "OK" in r.stdout, r.stdout + r.stderr
+    assert f"tile_n={bn} " in r.stderr and "ctas/mma=2" in r.stderr
