@@ -498,7 +498,7 @@ dg_status_t dg_m_grouped_fp8_gemm_nt_masked(const uint8_t *a, const float *sfa, 
     // columns (one FMA per element, no per-column scale traffic).  Groups with
     // fewer than 128 valid rows leave the other lanes idle; the weight stream,
     // which bounds this layout, is read once per token block.
-    // DG_MASKED_BN=128|256 overrides the tile width (tuning sweeps)
+    // DG_MASKED_BN=64|128|256 overrides the tile width (tuning sweeps)
     static const int forced_bn = [] {
         const char *e = std::getenv("DG_MASKED_BN");
         return e ? std::atoi(e) : 0;
@@ -507,9 +507,10 @@ dg_status_t dg_m_grouped_fp8_gemm_nt_masked(const uint8_t *a, const float *sfa, 
     // 256-wide grid ends in a long partial wave (measured 123 us vs 112 us on
     // 16 groups x N 4096); the weight stream is read once either way
     int bn = 128;
-    if (forced_bn == 128 || forced_bn == 256) bn = forced_bn;
+    if (forced_bn == 64 || forced_bn == 128 || forced_bn == 256) bn = forced_bn;
     if ((st = make_map(&ma, a, K, Mmax, G, 128)) != DG_SUCCESS) return st;
     if ((st = make_map(&mb, b, K, N, G, bn)) != DG_SUCCESS) return st;
+    if (bn == 64) return launch<64, false, 8, dg::kMasked>(ma, mb, md, p, grid, 1, 1, s);
     if (bn == 128) return launch<128, false, 6, dg::kMasked>(ma, mb, md, p, grid, 1, 1, s);
     return launch<256, false, 4, dg::kMasked>(ma, mb, md, p, grid, 1, 1, s);
 }

@@ -122,3 +122,25 @@ def test_dense_pair_tile_widths(bn):
     r = subprocess.run([sys.executable, "-c", code], env=env, capture_output=True, text=True, timeout=300)
     assert r.returncode == 0 and "OK" in r.stdout, r.stdout + r.stderr
     assert f"tile_n={bn} " in r.stderr and "ctas/mma=2" in r.stderr
+
+
+@pytest.mark.parametrize("bn", [64, 128, 256])
+def test_masked_tile_widths(bn):
+    """Every masked tile width (DG_MASKED_BN forces it, in a child process):
+    16 experts, Mmax 256, N 2112 (a weight tail), K 1024, whole output and the
+    untouched rows."""
+    import os, subprocess, sys
+    code = ("import sys; sys.path[:0] = [%r, %r]\n"
+            "import numpy as np, torch, workloads as W, oracle\n"
+            "from gpu_util import SENTINEL, DeviceProblem, compare, to_f64, valid_mask\n"
+            "p = W.make_masked_uniform(16, 256, 2112, 1024, seed=308)\n"
+            "dp = DeviceProblem(p); dp.fill_sentinel(); d = to_f64(dp.run())\n"
+            "compare(d, oracle.solve(p), valid_mask(p))\n"
+            "raw = dp.d.view(torch.int16).cpu().numpy()\n"
+            "assert all((raw[g, m:] == np.int16(SENTINEL)).all() for g, m in enumerate(p.masked_m))\n"
+            "print('OK')\n"
+            % (os.path.dirname(os.path.dirname(__file__)), os.path.dirname(__file__)))
+    env = dict(os.environ, DG_MASKED_BN=str(bn), DG_VERBOSE="1")
+    r = subprocess.run([sys.executable, "-c", code], env=env, capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0 and "OK" in r.stdout, r.stdout + r.stderr
+    assert f"tile_n={bn} " in r.stderr
