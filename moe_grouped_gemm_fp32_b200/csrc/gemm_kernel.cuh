@@ -867,9 +867,20 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
         int stage = 0, buf = 0, sslot = 0;
         uint32_t phase = 0, tphase = 0, sphase = 0;
         bool ok = true;
+        // contiguous layout: the next tile is decoded before this tile's epilogue,
+        // so its group-index loads from global memory overlap the stores
+        constexpr bool kDecodeAhead = kLayout == kContiguous;
+        Tile tl_ahead;
+        bool ahead_valid = false;
+        int t_ahead = -1;
         for (int t = t_first; ok && t < num_tiles; t += t_step) {
             Tile tl;
-            if (!TM::decode(t, p, prefix, tl)) continue;
+            if (kDecodeAhead && t == t_ahead) {
+                if (!ahead_valid) continue;
+                tl = tl_ahead;
+            } else if (!TM::decode(t, p, prefix, tl)) {
+                continue;
+            }
 #pragma unroll
             for (int i = 0; i < kHalf; ++i) acc[i] = 0.f;
             const int my_tok = tl.tok0 + my_row0 + lrow;   // normal mode: this thread's token row
@@ -1014,6 +1025,10 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
             last_nvalid = nvalid;
             have_tile = true;
             if (clustered) break;   // one tile; reduced below
+            if (kDecodeAhead && t + t_step < num_tiles) {
+                t_ahead = t + t_step;
+                ahead_valid = TM::decode(t_ahead, p, prefix, tl_ahead);
+            }
             // ------------------------------------------------ epilogue (direct)
             const size_t row_base = (kLayout == kMasked || kLayout == kKGrouped) ? static_cast<size_t>(tl.g) * p.M : 0;
             // the TMA store may write every row of this CTA's 128-row block:
