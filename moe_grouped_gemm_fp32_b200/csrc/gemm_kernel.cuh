@@ -610,7 +610,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
         if (ptx::elect_one()) {
             int stage = 0, sslot = 0;
             uint32_t phase = 0, sphase = 0;
-            long long issued = 0;
+            long long issued = 0, issued_s = 0;   // operand stages / swap-mode scale slots loaded
             bool ok = (p.debug_flags & kDebugProducerIdle) == 0;
             for (int t = t_first; ok && t < num_tiles; t += t_step) {
                 Tile tl;
@@ -636,9 +636,21 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
                 const int kb_lo = max(kb_begin, tl.kb0), kb_hi = min(kb_end, tl.kb1);
                 for (int kb = kb_lo; kb < kb_hi; ++kb) {
                     if (!wait(empty_bar(stage), phase ^ 1u, kSiteProducerEmpty)) { ok = false; break; }
-                    if (kSwap && !wait(sempty_bar(sslot), sphase ^ 1u, kSiteProducerEmpty)) { ok = false; break; }
                     const uint32_t sx = s_base + stage * L::kStageBytes;
                     const uint32_t sy = sx + L::kXBytes;
+                    if constexpr (kSwap) {
+                        // swap mode keeps the scales on their own barrier ring: the operand
+                        // loads go first (the first bytes of a decode-shaped GEMM are on its
+                        // critical path), then the scales once their slot is free
+                        ptx::mbar_arrive_expect_tx(full_bar(stage), op_bytes);
+                        ptx::tma_load_3d(sx, &tm_b, full_bar(stage), kb * kBlockK, tl.n0, tl.b_grp);
+                        for (int i = 0; i < nload; ++i)
+                            ptx::tma_load_3d(sy + i * kTokBox * kBlockK, &tm_a, full_bar(stage), kb * kBlockK,
+                                             tl.a_row + i * kTokBox, tl.a_grp);
+                        ++issued;
+                        if (++stage == kStages) { stage = 0; phase ^= 1u; }
+                        if (!wait(sempty_bar(sslot), sphase ^ 1u, kSiteProducerEmpty)) { ok = false; break; }
+                    }
                     const uint32_t slot = slot_base + (kSwap ? sslot : stage) * L::kSlotBytes;
                     const uint32_t scale_bar = kSwap ? sfull_bar(sslot) : full_bar(stage);
 #pragma unroll
@@ -650,20 +662,15 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
                             ptx::st_shared_f32(dst, 0.f);
                     }
                     ptx::cp_async_arrive(scale_bar);
-                    if (kSwap) {
-                        ptx::mbar_arrive_expect_tx(scale_bar, sa_bytes);
-                        ptx::mbar_arrive_expect_tx(full_bar(stage), op_bytes);
-                    } else {
-                        ptx::mbar_arrive_expect_tx(full_bar(stage), op_bytes + sa_bytes);
-                    }
+                    if (kSwap) ptx::mbar_arrive_expect_tx(scale_bar, sa_bytes);
+                    else ptx::mbar_arrive_expect_tx(full_bar(stage), op_bytes + sa_bytes);
                     if (sa_bytes)
                         ptx::bulk_load(slot, sfa_g + static_cast<size_t>(kb) * p.ld_sfa + sa_row0, sa_bytes,
                                        scale_bar);
                     if (kSwap) {
-                        ptx::tma_load_3d(sx, &tm_b, full_bar(stage), kb * kBlockK, tl.n0, tl.b_grp);
-                        for (int i = 0; i < nload; ++i)
-                            ptx::tma_load_3d(sy + i * kTokBox * kBlockK, &tm_a, full_bar(stage), kb * kBlockK,
-                                             tl.a_row + i * kTokBox, tl.a_grp);
+                        ++issued_s;
+                        if (++sslot == kSlots) { sslot = 0; sphase ^= 1u; }
+                        continue;
                     } else if (kPair) {
                         // both CTAs' operand bytes complete on the MMA CTA's barrier
                         const uint32_t fb = leader_addr(full_bar(stage));
@@ -676,7 +683,6 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
                     }
                     ++issued;
                     if (++stage == kStages) { stage = 0; phase ^= 1u; }
-                    if (kSwap && ++sslot == kSlots) { sslot = 0; sphase ^= 1u; }
                 }
             }
             // wind-down: never leave with TMA writes into this CTA's smem in flight
@@ -684,9 +690,9 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
             // cannot see its operand bytes land on its own barrier; for it the final
             // cluster barrier, reached only after the MMA CTA consumed every stage or
             // ran out of time waiting for it, covers them.
-            auto drain = [&](long long depth, auto bar_of) {
-                const long long first = issued > depth ? issued - depth : 0;
-                for (long long i = first; i < issued; ++i) {
+            auto drain = [&](long long depth, long long count, auto bar_of) {
+                const long long first = count > depth ? count - depth : 0;
+                for (long long i = first; i < count; ++i) {
                     const uint32_t bar = bar_of(static_cast<int>(i % depth));
                     const uint32_t par = static_cast<uint32_t>((i / depth) & 1);
                     const long long start = clock64();
@@ -698,8 +704,8 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
                     }
                 }
             };
-            drain(kStages, full_bar);
-            if constexpr (kSwap) drain(kSlots, sfull_bar);
+            drain(kStages, issued, full_bar);
+            if constexpr (kSwap) drain(kSlots, issued_s, sfull_bar);
         }
         __syncwarp();
     } else if (warp == 1) {
