@@ -149,10 +149,10 @@ namespace {
 using namespace dg_host;
 
 // D as a 2-D BF16 tensor {N, rows} (masked / K-grouped: all groups' rows
-// stacked), box {32 columns, 32 rows} with 64-byte swizzle: the TMA-store
-// epilogue's box.  A null d (no BF16 output) gives an all-zero map the kernel
+// stacked), box {32 columns, box_rows rows} with 64-byte swizzle: the TMA-store
+// epilogue's box (32 rows per warp; CTA pairs store 128-row boxes of a staged tile).  A null d (no BF16 output) gives an all-zero map the kernel
 // never uses.
-dg_status_t make_d_map(CUtensorMap *m, void *d, long long N, long long rows) {
+dg_status_t make_d_map(CUtensorMap *m, void *d, long long N, long long rows, int box_rows = 32) {
     std::memset(m, 0, sizeof(*m));
     if (!d || rows <= 0) return DG_SUCCESS;
     EncodeTiledFn fn = encode_fn();
@@ -163,7 +163,7 @@ dg_status_t make_d_map(CUtensorMap *m, void *d, long long N, long long rows) {
     }
     cuuint64_t dims[2] = {static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(rows)};
     cuuint64_t strides[1] = {static_cast<cuuint64_t>(N) * 2};
-    cuuint32_t box[2] = {32, 32};
+    cuuint32_t box[2] = {32, static_cast<cuuint32_t>(box_rows)};
     cuuint32_t estr[2] = {1, 1};
     CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, dims, strides, box, estr,
                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
@@ -181,6 +181,13 @@ dg_status_t make_d_map(CUtensorMap *m, void *d, long long N, long long rows) {
 dg_status_t make_map(CUtensorMap *m, const void *base, long long K, long long rows,
                      long long groups, int box_rows) {
     return make_kmajor_map(m, base, 1, K, rows, groups, box_rows);
+}
+
+// Row count of the D map's TMA-store box for a kernel instantiation: CTA-pair
+// kernels that stage the whole tile store 128-row boxes, the others 32 rows per warp.
+template <int kBN, int kStages, int kCtaGroup>
+constexpr int d_box_rows() {
+    return dg::SmemLayout<kBN, false, kStages, kCtaGroup>::kTileStaging ? dg::kTileX : 32;
 }
 
 // ------------------------------------------------------------------ validation
@@ -387,22 +394,27 @@ dg_status_t dg_fp8_gemm_nt(const uint8_t *a, const float *sfa, int ld_sfa, const
         return e ? std::atoi(e) : 0;
     }();
     const long long row_pairs = (M + 255) / 256;
-    const int pm224 = max_active_clusters<224, false, 6, dg::kDense, 2>(2);
+    const int pm224 = max_active_clusters<224, false, 5, dg::kDense, 2>(2);
     const int pm256 = max_active_clusters<256, false, 6, dg::kDense, 2>(2);
     int bn = pair_efficiency(row_pairs, N, 224, pm224) > pair_efficiency(row_pairs, N, 256, pm256) + 1e-9
                  ? 224 : 256;
     if (forced_bn == 128 || forced_bn == 160 || forced_bn == 224 || forced_bn == 256) bn = forced_bn;
-    const int pairs_max = bn == 128   ? max_active_clusters<128, false, 8, dg::kDense, 2>(2)
-                          : bn == 160 ? max_active_clusters<160, false, 7, dg::kDense, 2>(2)
+    const int pairs_max = bn == 128   ? max_active_clusters<128, false, 7, dg::kDense, 2>(2)
+                          : bn == 160 ? max_active_clusters<160, false, 6, dg::kDense, 2>(2)
                           : bn == 224 ? pm224 : pm256;
     if (pairs_max <= 0) return cuda_fail(cudaErrorInvalidConfiguration, "no resident CTA pair");
     const int tiles = ((M + 255) / 256) * ((N + bn - 1) / bn);
     const int pairs = tiles < pairs_max ? tiles : pairs_max;
+    {
+        const int box = bn == 128 ? d_box_rows<128, 7, 2>() : bn == 160 ? d_box_rows<160, 6, 2>()
+                        : bn == 224 ? d_box_rows<224, 5, 2>() : d_box_rows<256, 6, 2>();
+        if ((st = make_d_map(&md, d, N, M, box)) != DG_SUCCESS) return st;
+    }
     if ((st = make_map(&ma, a, K, M, 1, 128)) != DG_SUCCESS) return st;
     if ((st = make_map(&mb, b, K, N, 1, bn / 2)) != DG_SUCCESS) return st;
-    if (bn == 128) return launch<128, false, 8, dg::kDense, 2>(ma, mb, md, p, 2 * pairs, 1, 2, s);
-    if (bn == 160) return launch<160, false, 7, dg::kDense, 2>(ma, mb, md, p, 2 * pairs, 1, 2, s);
-    if (bn == 224) return launch<224, false, 6, dg::kDense, 2>(ma, mb, md, p, 2 * pairs, 1, 2, s);
+    if (bn == 128) return launch<128, false, 7, dg::kDense, 2>(ma, mb, md, p, 2 * pairs, 1, 2, s);
+    if (bn == 160) return launch<160, false, 6, dg::kDense, 2>(ma, mb, md, p, 2 * pairs, 1, 2, s);
+    if (bn == 224) return launch<224, false, 5, dg::kDense, 2>(ma, mb, md, p, 2 * pairs, 1, 2, s);
     return launch<256, false, 6, dg::kDense, 2>(ma, mb, md, p, 2 * pairs, 1, 2, s);
 }
 
@@ -438,7 +450,7 @@ dg_status_t dg_m_grouped_fp8_gemm_nt_contiguous(const uint8_t *a, const float *s
         // CTA pairs with 256-row tiles; pairs straddling a group boundary run
         // a second pass (the tile count grows by at most (G-1) x N-tiles)
         const long long row_pairs = (M_total / 128 + 1) / 2;
-        const int pm224 = max_active_clusters<224, false, 6, dg::kContiguous, 2>(2);
+        const int pm224 = max_active_clusters<224, false, 5, dg::kContiguous, 2>(2);
         const int pm256 = max_active_clusters<256, false, 6, dg::kContiguous, 2>(2);
         const int bn = pair_efficiency(row_pairs, N, 224, pm224) > pair_efficiency(row_pairs, N, 256, pm256) + 1e-9
                            ? 224 : 256;
@@ -446,9 +458,11 @@ dg_status_t dg_m_grouped_fp8_gemm_nt_contiguous(const uint8_t *a, const float *s
         if (pairs_max > 0) {
             const long long tiles = row_pairs * ((N + bn - 1) / bn);
             const int pairs = tiles < pairs_max ? static_cast<int>(tiles) : pairs_max;
+            const int box = bn == 224 ? d_box_rows<224, 5, 2>() : d_box_rows<256, 6, 2>();
+            if ((st = make_d_map(&md, d, N, M_total, box)) != DG_SUCCESS) return st;
             if ((st = make_map(&ma, a, K, M_total, 1, 128)) != DG_SUCCESS) return st;
             if ((st = make_map(&mb, b, K, N, G, bn / 2)) != DG_SUCCESS) return st;
-            if (bn == 224) return launch<224, false, 6, dg::kContiguous, 2>(ma, mb, md, p, 2 * pairs, 1, 2, s);
+            if (bn == 224) return launch<224, false, 5, dg::kContiguous, 2>(ma, mb, md, p, 2 * pairs, 1, 2, s);
             return launch<256, false, 6, dg::kContiguous, 2>(ma, mb, md, p, 2 * pairs, 1, 2, s);
         }
     }
@@ -547,7 +561,7 @@ dg_status_t dg_k_grouped_fp8_gemm_nt_contiguous(const uint8_t *a, const float *s
     }
     // CTA pairs: 256 x bn tiles (tcgen05.mma.cta_group::2), as for large dense GEMMs
     const long long row_pairs = static_cast<long long>(G) * ((M + 255) / 256);
-    const int pm224 = max_active_clusters<224, false, 6, dg::kKGrouped, 2>(2);
+    const int pm224 = max_active_clusters<224, false, 5, dg::kKGrouped, 2>(2);
     const int pm256 = max_active_clusters<256, false, 6, dg::kKGrouped, 2>(2);
     const int bn = pair_efficiency(row_pairs, N, 224, pm224) > pair_efficiency(row_pairs, N, 256, pm256) + 1e-9
                        ? 224 : 256;
@@ -555,8 +569,10 @@ dg_status_t dg_k_grouped_fp8_gemm_nt_contiguous(const uint8_t *a, const float *s
     if (pairs_max <= 0) return cuda_fail(cudaErrorInvalidConfiguration, "no resident CTA pair");
     const long long tiles = row_pairs * ((N + bn - 1) / bn);
     const int pairs = tiles < pairs_max ? static_cast<int>(tiles) : pairs_max;
+    const int box = bn == 224 ? d_box_rows<224, 5, 2>() : d_box_rows<256, 6, 2>();
+    if ((st = make_d_map(&md, d, N, static_cast<long long>(G) * M, box)) != DG_SUCCESS) return st;
     if ((st = make_map(&mb, b, K, N, 1, bn / 2)) != DG_SUCCESS) return st;
-    if (bn == 224) return launch<224, false, 6, dg::kKGrouped, 2>(ma, mb, md, p, 2 * pairs, 1, 2, s);
+    if (bn == 224) return launch<224, false, 5, dg::kKGrouped, 2>(ma, mb, md, p, 2 * pairs, 1, 2, s);
     return launch<256, false, 6, dg::kKGrouped, 2>(ma, mb, md, p, 2 * pairs, 1, 2, s);
 }
 

@@ -364,7 +364,14 @@ struct SmemLayout {
     // (64-byte rows, 64B swizzle) for the TMA-store epilogue
     static constexpr int kOutBoxBytes = 32 * 64;
     static constexpr int kOutOffset = (kRecvOffset + kRecvBytes + 1023) / 1024 * 1024;
-    static constexpr int kOutBytes = kSwap ? 0 : 8 * kOutBoxBytes;
+    // CTA pairs stage a whole finished tile instead (this CTA's 128 rows x kBN
+    // columns of BF16, as kBN/32 boxes of 128 rows x 32 columns, 64B swizzle) and
+    // one thread stores it, so the promotion warps never wait for the stores
+    // (where it fits next to the pipeline stages; otherwise per-warp boxes)
+    static constexpr int kStageBoxBytes = kTileX * 64;
+    static constexpr bool kTileStaging =
+        !kSwap && kCtaGroup == 2 && kOutOffset + (kBN / 32) * kStageBoxBytes + 1024 <= 227 * 1024;
+    static constexpr int kOutBytes = kTileStaging ? (kBN / 32) * kStageBoxBytes : (kSwap ? 0 : 8 * kOutBoxBytes);
     static constexpr int kUsed = kOutOffset + kOutBytes;
     static constexpr int kAlloc = (kUsed + 1024 > kMinSmem) ? kUsed + 1024 : kMinSmem;
     static constexpr int kTmemCols = kAccBufs * kBN <= 32    ? 32
@@ -378,6 +385,7 @@ struct SmemLayout {
     static_assert(kPrefixOffset % 16 == 0, "prefix table alignment");
     static_assert(kRecvOffset % 16 == 0, "split-K pushes and reads are 16-byte vectors");
     static_assert(kOutOffset % 1024 == 0, "swizzled TMA-store boxes need aligned shared memory");
+    static_assert(!kTileStaging || kBN % 32 == 0, "tile staging stores 32-column boxes");
     static_assert(kAlloc <= 227 * 1024, "shared memory budget");
 };
 
@@ -1085,6 +1093,40 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
                         *reinterpret_cast<uint4 *>(qrow + c) = make_uint4(w[0], w[1], w[2], w[3]);
                     }
                     if (half == 0) p.s_out[static_cast<size_t>(ablk) * p.ld_s_out + row_base + my_tok] = sc;
+                }
+            } else if (L::kTileStaging && tma_epilogue) {
+                // CTA pairs: the whole tile is staged as BF16 (box c = tile columns
+                // [32c, 32c + 32), 128 rows of 64 bytes, 64B swizzle) and one thread
+                // issues the boxes' TMA stores; the warps go on to the next tile at
+                // once.  The staging of the previous tile must have been read first.
+                const bool issuer = warp == kPromoWarp0 && lane == 0;
+                if (issuer) ptx::bulk_wait_read0();
+                ptx::named_bar_sync(3, 256);
+                uint8_t *stg = smem + L::kOutOffset;
+                const int sw = (lrow >> 1) & 3;                    // 64B swizzle of this row
+#pragma unroll
+                for (int j = 0; j < kHalf; j += 8) {
+                    const int col = out_col(j);                    // tile column (a multiple of 8)
+                    __nv_bfloat162 h0 = __floats2bfloat162_rn(acc[j + 0], acc[j + 1]);
+                    __nv_bfloat162 h1 = __floats2bfloat162_rn(acc[j + 2], acc[j + 3]);
+                    __nv_bfloat162 h2 = __floats2bfloat162_rn(acc[j + 4], acc[j + 5]);
+                    __nv_bfloat162 h3 = __floats2bfloat162_rn(acc[j + 6], acc[j + 7]);
+                    const int q = (col & 31) >> 3;                 // 16-byte chunk within the box row
+                    *reinterpret_cast<uint4 *>(stg + (col >> 5) * L::kStageBoxBytes + lrow * 64 + ((q ^ sw) << 4)) =
+                        make_uint4(*reinterpret_cast<uint32_t *>(&h0), *reinterpret_cast<uint32_t *>(&h1),
+                                   *reinterpret_cast<uint32_t *>(&h2), *reinterpret_cast<uint32_t *>(&h3));
+                }
+                ptx::fence_proxy_async_smem();
+                ptx::named_bar_sync(3, 256);
+                if (issuer) {
+                    const int drow0 = static_cast<int>(row_base) + tl.tok0 + my_row0;
+#pragma unroll 1
+                    for (int c = 0; c < kBN / 32; ++c) {
+                        const int col0 = tl.n0 + 32 * c;
+                        if (col0 < p.N)
+                            ptx::tma_store_2d(&tm_d, ptx::smem_u32(stg + c * L::kStageBoxBytes), col0, drow0);
+                    }
+                    ptx::bulk_commit();
                 }
             } else if (!kSwap && tma_epilogue) {
                 // TMA-store epilogue: each warp converts its 32 rows x 32 columns
