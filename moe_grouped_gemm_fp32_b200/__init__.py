@@ -25,6 +25,8 @@ LIB_PATH = os.path.join(_HERE, "_dg.so")
 HEADER = os.path.join(os.path.dirname(_HERE), "include", "dg.h")
 
 DG_SUCCESS = 0
+# size of the fixed device array of dg_m_grouped_fp8_ffn_contiguous_noalloc (DG_NOALLOC_SCRATCH_BYTES)
+NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
 STATUS_NAMES = {0: "DG_SUCCESS", 1: "DG_ERR_INVALID_VALUE", 2: "DG_ERR_MISALIGNED",
                 3: "DG_ERR_UNSUPPORTED_SHAPE", 4: "DG_ERR_UNSUPPORTED_DEVICE",
                 5: "DG_ERR_CUDA", 6: "DG_ERR_TIMEOUT"}

@@ -89,6 +89,22 @@ def test_grouped_validation(L):
     assert L.dg_m_grouped_bf16_gemm_nt_masked(FAKE, FAKE, FAKE, FAKE, 1024, big, 256, 512, None) == 3
 
 
+def test_no_alloc_ffn_refuses_before_any_device_work(L):
+    """The fused FFN without allocation checks its fixed array's limit (16 MiB:
+    codes M_total * I, 256-byte rounded, plus (I / 128) scale rows of M_total
+    rounded to 4 floats) and its shape rules before touching a device."""
+    f = L.dg_m_grouped_fp8_ffn_contiguous_noalloc
+    args = lambda M, H, I, G: (FAKE, FAKE, max(M, 4), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, M, H, I, G, None)
+    assert f(*args(-1, 256, 256, 1)) == 1                 # negative M_total
+    assert f(*args(128, 256, 200, 1)) == 3                # I not a multiple of 128
+    assert f(*args(8192, 256, 2048, 1)) == 3              # 16 MiB of codes plus scales: too large
+    assert f(*args(7936, 256, 2048, 1)) == 4              # fits (15.5 MiB + 0.5 MiB): no device here
+    assert 8192 * 2048 + 16 * 8192 * 4 > dg.NOALLOC_SCRATCH_BYTES >= 7936 * 2048 + 16 * 7936 * 4
+    import re
+    m = re.search(r"#define DG_NOALLOC_SCRATCH_BYTES \((\d+)u \* 1024u \* 1024u\)", open(dg.HEADER).read())
+    assert m and int(m.group(1)) * 1024 * 1024 == dg.NOALLOC_SCRATCH_BYTES
+
+
 def test_python_binding_rejects_cpu_tensors():
     import torch
     a = torch.zeros((64, 128), dtype=torch.uint8)
