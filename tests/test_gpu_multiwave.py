@@ -144,3 +144,46 @@ def test_masked_tile_widths(bn):
     r = subprocess.run([sys.executable, "-c", code], env=env, capture_output=True, text=True, timeout=300)
     assert r.returncode == 0 and "OK" in r.stdout, r.stdout + r.stderr
     assert f"tile_n={bn} " in r.stderr
+
+
+# ------------------------------------------------------------------ BF16 GEMMs past one wave
+def _bf16_run_and_ref(prob):
+    t = lambda bits: torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).cuda()
+    a, b = t(prob.a), t(prob.b)
+    d = torch.empty(prob.d_shape(), dtype=torch.bfloat16, device="cuda")
+    d.view(torch.int16).fill_(SENTINEL)
+    if prob.layout == "dense":
+        dg.dg_bf16_gemm_nt(a, b[0], d)
+    elif prob.layout == "contiguous":
+        dg.dg_m_grouped_bf16_gemm_nt_contiguous(a, b, d, torch.from_numpy(prob.m_indices).cuda())
+    else:
+        dg.dg_m_grouped_bf16_gemm_nt_masked(a, b, d, torch.from_numpy(prob.masked_m).cuda())
+    torch.cuda.synchronize()
+    ref = oracle.gemm_bf16(prob.layout, prob.a, prob.b[0] if prob.layout == "dense" else prob.b,
+                           prob.M, prob.N, prob.K, G=prob.G, m_indices=prob.m_indices, masked_m=prob.masked_m)
+    return d, ref
+
+
+def test_bf16_dense_several_waves():
+    # 2048 x 4096 x 1024: 16 token blocks x 16-19 weight tiles on 148 CTAs, the two
+    # TMEM accumulators rotating over ~2 tiles per CTA
+    prob = W.make_bf16_dense(2048, 4096, 1024, seed=401)
+    d, ref = _bf16_run_and_ref(prob)
+    compare(to_f64(d), ref, np.ones(ref.shape, bool))
+
+
+def test_bf16_contiguous_several_waves():
+    prob = W.make_bf16_contiguous([700, 0, 1100, 513, 257, 900], 2048, 1024, seed=402)
+    d, ref = _bf16_run_and_ref(prob)
+    compare(to_f64(d), ref, np.broadcast_to((prob.m_indices >= 0)[:, None], prob.d_shape()))
+
+
+def test_bf16_masked_several_waves():
+    rng = np.random.default_rng(403)
+    masked_m = rng.integers(0, 257, size=16)
+    prob = W.make_bf16_masked(masked_m.tolist(), 256, 2048, 1024, seed=403)
+    d, ref = _bf16_run_and_ref(prob)
+    rows = np.arange(256)[None, :] < prob.masked_m[:, None]
+    valid = np.broadcast_to(rows[:, :, None], prob.d_shape())
+    compare(to_f64(d), ref, valid)
+    assert (d.view(torch.int16).cpu().numpy()[~valid] == np.int16(SENTINEL)).all()
