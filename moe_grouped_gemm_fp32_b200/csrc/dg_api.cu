@@ -301,7 +301,9 @@ int max_active_clusters(int cluster_x) {
 
 // Split-K factor for swap-mode tiles: the largest split <= 8 such that every
 // cluster of the grid is resident at once (one wave), each CTA keeps at least
-// two K-blocks, and the CTAs fit on the SMs.  DG_SPLIT_K overrides it (tuning).
+// four K-blocks, and the CTAs fit on the SMs.  The cluster exchange costs about
+// 3 us, more than streaming a few K-blocks saves: 128 x 256 x 512 ran 7.9 us
+// per call unsplit against 9.1 us split in two.  DG_SPLIT_K overrides it (tuning).
 template <int kBN, int kStages, int kLayout>
 int choose_split(int tiles, int num_kb, int num_sms) {
     static int forced = [] {
@@ -310,7 +312,7 @@ int choose_split(int tiles, int num_kb, int num_sms) {
     }();
     if (forced >= 1 && forced <= 8) return num_kb >= 2 * forced ? forced : 1;
     for (int split = 8; split >= 2; --split) {
-        if (tiles * split > num_sms || num_kb < 2 * split) continue;
+        if (tiles * split > num_sms || num_kb < 4 * split) continue;
         if (max_active_clusters<kBN, true, kStages, kLayout>(split) >= tiles) return split;
     }
     return 1;

@@ -827,8 +827,9 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
     // (warps kPromoWarp0 and up)
     //
     // Column ownership.  Normal mode: warpgroup h owns the contiguous columns
-    // [h*kHalf, (h+1)*kHalf); each chunk of kChunk columns lies inside one
-    // 128-row weight block, whose scale the chunk uses.  Swap mode: columns
+    // [h*kHalf, (h+1)*kHalf) (224-wide tiles: alternate 32-column rounds, see
+    // round_col); every 16-column group lies inside one 128-row weight block,
+    // whose scale it uses.  Swap mode: columns
     // are tokens and the tile may hold fewer than kBN of them, so the chunks
     // are dealt alternately (chunk 2c+h to warpgroup h) to keep both
     // warpgroups busy; chunks past the tile's token count are skipped.

@@ -190,6 +190,25 @@ def test_default_run_is_the_contiguous_prefill_with_every_shape(monkeypatch, cap
     assert line["measurement"]["launch_floor_ms"] == 0.006
 
 
+def test_rotating_graph_copies_exceed_twice_the_l2():
+    """Decode-sized inputs get enough copies that together they exceed twice the
+    L2, so every call of the rotating-graph timing reads from HBM; small and
+    large inputs are not timed that way."""
+    for w in ("dense_decode_m64", "dense_decode_m128"):
+        prob = bench.rank_problem(w, 0)
+        nbytes = sum(x.nbytes for x in (prob.a, prob.sfa, prob.b, prob.sfb))   # the call's host inputs
+        sets = bench.rotation_sets(nbytes)
+        assert sets >= 2 and (sets - 1) * nbytes > 2 * bench.L2_BYTES
+    assert bench.rotation_sets(264224) == 0
+    assert bench.rotation_sets(500 << 20) == 0
+    t = bench.Timing("dense_decode_m64", bench.rank_problem("dense_decode_m64", 0), 0.015, 0.015, 1,
+                     graph_ms=0.0105, graph_sets=18, graph_calls=50)
+    e = bench.shape_entry(t, 1)["graph_rotating"]
+    assert e["unit"] == "GB/s" and e["input_copies"] == 18 and e["ms_per_call"] == 0.0105
+    assert abs(e["value"] - t.prob.bytes() / 0.0105e-3 / 1e9) < 1e-6 * e["value"]
+    assert "vs_pages" in e
+
+
 def test_shape_selection():
     assert bench.parse_shapes("auto", "contiguous_g4") == list(bench.SHAPES)
     assert bench.parse_shapes("auto", "dense_large") == []
