@@ -1027,6 +1027,8 @@ def main():
         line["graph"] = {"value": metric_value(prob, unit, graph_ms, world), "unit": unit,
                          "ms_per_call": graph_ms, "calls_per_graph": GRAPH_CALLS,
                          "l2": "not flushed between calls (B alone exceeds L2)"}
+    if head.graph_ms > 0:
+        line["graph_rotating"] = shape_entry(head, world)["graph_rotating"]
     if shapes:
         line["shapes"] = {t.workload: shape_entry(t, world) for t in shapes}
     if not args.no_cpu_baseline and world == 1:

@@ -209,6 +209,22 @@ def test_rotating_graph_copies_exceed_twice_the_l2():
     assert "vs_pages" in e
 
 
+def test_headline_carries_its_rotating_graph_figure(monkeypatch, capsys):
+    """A decode-sized headline (``--workload dense_decode_m64 --shapes none``)
+    prints its rotating-graph figure at the top level."""
+    prob = bench.rank_problem("dense_decode_m64", 0)
+    head = bench.Timing("dense_decode_m64", prob, 0.015, 0.015, 1, graph_ms=0.0104, graph_sets=18, graph_calls=50)
+    monkeypatch.setattr(bench, "run_ours", lambda a, r, w, lr: (head, 0.05, 10, 10, 0.0, [],
+                                                                 {"sm_mhz": 1965, "sm_max_mhz": 1965,
+                                                                  "reasons": []}, 0.0))
+    monkeypatch.setattr(sys, "argv", ["bench.py", "--workload", "dense_decode_m64", "--shapes", "none",
+                                      "--steps", "5", "--warmup", "3", "--no-cpu-baseline"])
+    assert bench.main() == 0
+    line = json.loads(capsys.readouterr().out.strip())
+    assert line["graph_rotating"]["ms_per_call"] == 0.0104
+    assert line["graph_rotating"]["value"] > line["value"]
+
+
 def test_shape_selection():
     assert bench.parse_shapes("auto", "contiguous_g4") == list(bench.SHAPES)
     assert bench.parse_shapes("auto", "dense_large") == []
