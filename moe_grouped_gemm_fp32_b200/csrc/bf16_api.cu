@@ -43,11 +43,11 @@ dg::Params bf16_params(void *d, int rows, int N, int K, int G, const DeviceInfo 
     return p;
 }
 
-template <int kBN, int kStages, int kLayout, bool kSplitK = false>
+template <int kBN, int kStages, int kLayout, bool kSplitK = false, int kCtaGroup = 1>
 dg_status_t launch_bf16(const CUtensorMap &ma, const CUtensorMap &mb, const dg::Params &p, int grid,
                         cudaStream_t stream, int grid_y = 1, int cluster_x = 1) {
-    using L = dg::Bf16Smem<kBN, kStages, kSplitK>;
-    auto kernel = dg::bf16_gemm_kernel<kBN, kStages, kLayout, kSplitK>;
+    using L = dg::Bf16Smem<kBN, kStages, kSplitK, kCtaGroup>;
+    auto kernel = dg::bf16_gemm_kernel<kBN, kStages, kLayout, kSplitK, kCtaGroup>;
     // one-time per-device set-up (idempotent; the atomic flag keeps racing first calls defined)
     static std::atomic<bool> configured[kMaxDevices] = {};
     int dev = 0;
@@ -58,8 +58,8 @@ dg_status_t launch_bf16(const CUtensorMap &ma, const CUtensorMap &mb, const dg::
         configured[dev].store(true, std::memory_order_release);
     }
     if (verbose())
-        std::fprintf(stderr, "[dg] bf16_gemm layout=%d bn=%d stages=%d grid=%dx%d cluster=%d split=%d smem=%d\n",
-                     kLayout, kBN, kStages, grid, grid_y, cluster_x, p.split, L::kAlloc);
+        std::fprintf(stderr, "[dg] bf16_gemm layout=%d bn=%d stages=%d ctas/mma=%d grid=%dx%d cluster=%d split=%d smem=%d\n",
+                     kLayout, kBN, kStages, kCtaGroup, grid, grid_y, cluster_x, p.split, L::kAlloc);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid, grid_y, 1);
     cfg.blockDim = dim3(dg::kBf16Threads, 1, 1);
@@ -92,11 +92,12 @@ int pick_bn(long long token_blocks, int N, int num_sms) {
     return eff(224) > eff(256) + 1e-9 ? 224 : 256;
 }
 
-// Resident clusters of `split` CTAs of the split-K kernel (0 if the query fails).
-template <int kBN, int kStages>
+// Resident clusters of `split` CTAs of the split-K kernel, or of CTA pairs of
+// the pair kernel (0 if the query fails).
+template <int kBN, int kStages, int kLayout = dg::kDense, bool kSplitK = true, int kCtaGroup = 1>
 int bf16_max_clusters(int split) {
-    using L = dg::Bf16Smem<kBN, kStages, true>;
-    auto kernel = dg::bf16_gemm_kernel<kBN, kStages, dg::kDense, true>;
+    using L = dg::Bf16Smem<kBN, kStages, kSplitK, kCtaGroup>;
+    auto kernel = dg::bf16_gemm_kernel<kBN, kStages, kLayout, kSplitK, kCtaGroup>;
     // per-device cache of an idempotent query (atomic: concurrent first calls are defined)
     static std::atomic<int> cache[kMaxDevices][9] = {};
     int dev = 0;
@@ -127,9 +128,55 @@ int bf16_max_clusters(int split) {
     return n;
 }
 
+// CTA pairs (256-row tiles, tcgen05.mma.cta_group::2) for the dense and
+// contiguous layouts with N > 128 and at least two 128-row blocks: each SM then
+// reads half of the weight tile per K-block.  DG_BF16_PAIRS=0 / =1 forces
+// single-CTA tiles / pairs (comparisons and tests).
+int bf16_pairs_env() {
+    static const int v = [] {
+        const char *e = std::getenv("DG_BF16_PAIRS");
+        return e ? (e[0] == '1' ? 1 : 0) : -1;
+    }();
+    return v;
+}
+
+template <int kLayout>
+dg_status_t dispatch_pairs(const CUtensorMap &ma, const void *b, int N, int K, int G, const dg::Params &p,
+                           long long row_pairs, cudaStream_t s, bool *done) {
+    *done = false;
+    const int pm224 = bf16_max_clusters<224, 6, kLayout, false, 2>(2);
+    const int pm256 = bf16_max_clusters<256, 6, kLayout, false, 2>(2);
+    auto eff = [&](int bn, int pairs_max) {
+        if (pairs_max <= 0) return 0.0;
+        const long long nt = (N + bn - 1) / bn;
+        const long long tiles = row_pairs * nt;
+        const long long waves = (tiles + pairs_max - 1) / pairs_max;
+        return (static_cast<double>(N) / (nt * bn)) * (static_cast<double>(tiles) / (waves * pairs_max));
+    };
+    const int bn = eff(224, pm224) > eff(256, pm256) + 1e-9 ? 224 : 256;
+    const int pairs_max = bn == 224 ? pm224 : pm256;
+    if (pairs_max <= 0) return DG_SUCCESS;   // no resident pair: the caller takes single-CTA tiles
+    CUtensorMap mb;
+    dg_status_t st = make_kmajor_map(&mb, b, 2, K, N, G, bn / 2);
+    if (st != DG_SUCCESS) return st;
+    const long long tiles = row_pairs * ((N + bn - 1) / bn);
+    const int pairs = tiles < pairs_max ? static_cast<int>(tiles) : pairs_max;
+    *done = true;
+    if (bn == 224) return launch_bf16<224, 6, kLayout, false, 2>(ma, mb, p, 2 * pairs, s, 1, 2);
+    return launch_bf16<256, 6, kLayout, false, 2>(ma, mb, p, 2 * pairs, s, 1, 2);
+}
+
 template <int kLayout>
 dg_status_t dispatch(const CUtensorMap &ma, const void *b, int N, int K, int G, const dg::Params &p,
                      long long tiles_hint_blocks, int grid_cap, cudaStream_t s) {
+    if constexpr (kLayout != dg::kMasked) {
+        if (N > 128 && bf16_pairs_env() != 0 && (tiles_hint_blocks >= 2 || bf16_pairs_env() == 1) &&
+            (kLayout != dg::kContiguous || G < dg::kMaxGroups)) {
+            bool done = false;
+            const dg_status_t st = dispatch_pairs<kLayout>(ma, b, N, K, G, p, (tiles_hint_blocks + 1) / 2, s, &done);
+            if (st != DG_SUCCESS || done) return st;
+        }
+    }
     const int bn = pick_bn(tiles_hint_blocks, N, grid_cap);
     CUtensorMap mb;
     dg_status_t st = make_kmajor_map(&mb, b, 2, K, N, G, bn);

@@ -19,6 +19,16 @@
 //   warps 4..7  epilogue: tcgen05.ld of the accumulator in 32-column chunks,
 //               BF16 round-to-nearest-even, 16-byte stores of each row.
 //
+// CTA pairs (kCtaGroup == 2; dense and contiguous layouts with many tiles): a
+// cluster of 2 CTAs computes one 256 x kBN tile with tcgen05.mma.cta_group::2.
+// Each CTA stages its own 128 token rows and half of the tile's weight rows, so
+// a K-block costs each SM 16 KB + kBN/2 x 128 B of shared memory and of L2 reads
+// instead of 16 KB + kBN x 128 B: the weight operand, which bounds single-CTA
+// tiles' shared-memory reads, is halved.  The even CTA issues the MMAs; both
+// CTAs' TMA bytes complete on its barrier, the MMA completions are multicast to
+// both CTAs, and each CTA's epilogue drains its own 128 accumulator rows and
+// releases the accumulator on the even CTA's barrier.
+//
 // Every wait is bounded (BoundedWait): on timeout the kernel records
 // DG_ERR_TIMEOUT in the device status word and winds down instead of hanging.
 #pragma once
@@ -36,10 +46,10 @@ __host__ __device__ constexpr uint32_t bf16_idesc(int m, int n) {
            (static_cast<uint32_t>(m >> 4) << 24);
 }
 
-template <int kBN, int kStages, bool kSplitK = false>
+template <int kBN, int kStages, bool kSplitK = false, int kCtaGroup = 1>
 struct Bf16Smem {
     static constexpr int kXBytes = kTileX * 128;        // 128 rows x 64 BF16
-    static constexpr int kYBytes = kBN * 128;
+    static constexpr int kYBytes = kBN / kCtaGroup * 128;   // this CTA's weight rows
     static constexpr int kStageBytes = kXBytes + kYBytes;
     static constexpr int kAccBufs = 2;
     static constexpr int kBarOffset = kStages * kStageBytes;
@@ -62,13 +72,16 @@ struct Bf16Smem {
                   "split-K staging lives in the operand stages");
 };
 
-template <int kBN, int kStages, int kLayout, bool kSplitK = false>
+template <int kBN, int kStages, int kLayout, bool kSplitK = false, int kCtaGroup = 1>
 __global__ void __launch_bounds__(kBf16Threads, 1)
 bf16_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                  const Params p) {
-    using L = Bf16Smem<kBN, kStages, kSplitK>;
+    using L = Bf16Smem<kBN, kStages, kSplitK, kCtaGroup>;
     static_assert(!kSplitK || kLayout == kDense, "split-K: dense layout");
-    using TM = TileMap<kBN, false, kLayout, 1>;
+    constexpr bool kPair = kCtaGroup == 2;
+    static_assert(!kPair || ((kLayout == kDense || kLayout == kContiguous) && !kSplitK),
+                  "CTA pairs: dense or contiguous, no split-K");
+    using TM = TileMap<kBN, false, kLayout, kCtaGroup>;
     static_assert(kBN == 128 || kBN == 224 || kBN == 256, "tile N");
     static_assert(kLayout != kKGrouped, "BF16: dense, contiguous and masked layouts");
     constexpr int kAccBufs = L::kAccBufs;
@@ -92,6 +105,10 @@ bf16_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant
     const int warp = threadIdx.x / 32;
     const int lane = threadIdx.x % 32;
     const BoundedWait wait{abort_flag, p.status, p.timeout_cycles};
+    // CTA pair: rank 0 issues the MMAs; its barriers count both CTAs' operand bytes
+    const uint32_t pair_rank = kPair ? (ptx::cluster_rank() & 1u) : 0u;
+    const bool mma_cta = pair_rank == 0;
+    auto leader_addr = [&](uint32_t local) { return kPair ? ptx::map_cluster(local, 0) : local; };
 
     if (threadIdx.x == 0) {
         ptx::prefetch_tmap(&tm_a);
@@ -102,7 +119,7 @@ bf16_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant
         }
         for (int b = 0; b < kAccBufs; ++b) {
             ptx::mbar_init(tfull_bar(b), 1);
-            ptx::mbar_init(tempty_bar(b), 4);          // one arrival per epilogue warp
+            ptx::mbar_init(tempty_bar(b), 4 * kCtaGroup);   // one arrival per epilogue warp of the pair
         }
         ptx::mbar_init(mma_done_bar, 1);
         ptx::mbar_init(recv_bar, 1);               // split-K: the owner's expect-tx arrival
@@ -135,22 +152,57 @@ bf16_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant
         }
         if (lane == 0) prefix[p.G] = carry;
     }
+    if (TM::kPairedGroups && warp == kEpiWarp0) {
+        // contiguous layout on CTA pairs: the pairs of 128-row blocks whose groups
+        // differ get a second pass (the tile scheduler lists them after the first
+        // passes); the table of such pairs, as in the FP8 kernel
+        const int nblk = p.M / kTileX, npairs = (nblk + 1) / 2;
+        int count = 0;
+        for (int base = 0; base < npairs; base += 32) {
+            const int pr = base + lane;
+            bool second = false;
+            if (pr < npairs) {
+                for (int b = 2 * pr; b <= 2 * pr + 1 && b < nblk; ++b)
+                    if (__ldg(p.m_indices + static_cast<size_t>(b) * kTileX) >= p.G)
+                        record_status(p.status, kStatusInvalid, kSiteBadGroup);
+                const int g0 = TM::block_group(p, 2 * pr), g1 = TM::block_group(p, 2 * pr + 1);
+                second = g0 >= 0 && g1 >= 0 && g0 != g1;
+            }
+            const unsigned ballot = __ballot_sync(0xffffffffu, second);
+            const int slot = count + __popc(ballot & ((1u << lane) - 1u));
+            if (second && slot < kMaxGroups) prefix[slot] = pr;
+            count += __popc(ballot);
+        }
+        if (count > kMaxGroups) {
+            if (lane == 0) record_status(p.status, kStatusInvalid, kSiteBadGroup);
+            count = kMaxGroups;
+        }
+        if (lane == 0) prefix[kMaxGroups] = count;
+    }
     if (warp == 1) {
-        ptx::tmem_alloc(ptx::smem_u32(tmem_slot), L::kTmemCols);
-        ptx::tmem_relinquish();
+        if constexpr (kPair) {
+            ptx::tmem_alloc_pair(ptx::smem_u32(tmem_slot), L::kTmemCols);
+            ptx::tmem_relinquish_pair();
+        } else {
+            ptx::tmem_alloc(ptx::smem_u32(tmem_slot), L::kTmemCols);
+            ptx::tmem_relinquish();
+        }
     }
     ptx::tc_fence_before();
     __syncthreads();
+    if constexpr (kPair) ptx::cluster_sync_all();   // the peer's barriers exist before any remote use
     ptx::tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+    // this CTA's token rows inside a pair tile
+    const int my_row0 = kPair ? static_cast<int>(pair_rank) * kTileX : 0;
 
     // split-K (dense, few tiles): a cluster of p.split CTAs shares one tile, each
     // CTA takes a contiguous range of K-blocks; the FP32 partials are summed in
     // rank order through distributed shared memory (see the epilogue)
     const bool clustered = kSplitK && p.split > 1;
     const int num_tiles = clustered ? static_cast<int>(gridDim.y) : TM::count(p, prefix);
-    const int t_first = clustered ? static_cast<int>(blockIdx.y) : static_cast<int>(blockIdx.x);
-    const int t_step = clustered ? num_tiles : static_cast<int>(gridDim.x);
+    const int t_first = clustered ? static_cast<int>(blockIdx.y) : static_cast<int>(blockIdx.x) / kCtaGroup;
+    const int t_step = clustered ? num_tiles : static_cast<int>(gridDim.x) / kCtaGroup;
     int kb_begin = 0, kb_end = p.num_kb;
     if (clustered) {
         // every CTA's receive barrier exists before another CTA signals it (its
@@ -179,16 +231,28 @@ bf16_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant
                 for (int kb = kb_begin; kb < kb_end; ++kb) {
                     if (!wait(empty_bar(stage), phase ^ 1u, kSiteProducerEmpty)) { ok = false; break; }
                     const uint32_t sx = s_base + stage * L::kStageBytes;
-                    ptx::mbar_arrive_expect_tx(full_bar(stage), L::kStageBytes);
-                    ptx::tma_load_3d(sx, &tm_a, full_bar(stage), kb * kBf16BlockK, tl.a_row, tl.a_grp);
-                    ptx::tma_load_3d(sx + L::kXBytes, &tm_b, full_bar(stage), kb * kBf16BlockK, tl.n0,
-                                     tl.b_grp);
+                    if constexpr (kPair) {
+                        // both CTAs' bytes complete on the MMA CTA's barrier
+                        if (mma_cta) ptx::mbar_arrive_expect_tx(full_bar(stage), 2u * L::kStageBytes);
+                        const uint32_t fb = leader_addr(full_bar(stage));
+                        ptx::tma_load_3d_pair(sx, &tm_a, fb, kb * kBf16BlockK, tl.a_row + my_row0, tl.a_grp);
+                        ptx::tma_load_3d_pair(sx + L::kXBytes, &tm_b, fb, kb * kBf16BlockK,
+                                              tl.n0 + static_cast<int>(pair_rank) * (kBN / 2), tl.b_grp);
+                    } else {
+                        ptx::mbar_arrive_expect_tx(full_bar(stage), L::kStageBytes);
+                        ptx::tma_load_3d(sx, &tm_a, full_bar(stage), kb * kBf16BlockK, tl.a_row, tl.a_grp);
+                        ptx::tma_load_3d(sx + L::kXBytes, &tm_b, full_bar(stage), kb * kBf16BlockK, tl.n0,
+                                         tl.b_grp);
+                    }
                     ++issued;
                     if (++stage == kStages) { stage = 0; phase ^= 1u; }
                 }
             }
-            // never leave with TMA writes into shared memory in flight
-            const long long first = issued > kStages ? issued - kStages : 0;
+            // never leave with TMA writes into shared memory in flight.  A pair's
+            // second CTA cannot see its bytes land on its own barrier; for it the
+            // final cluster barrier, reached only after the MMA CTA consumed every
+            // stage (or ran out of time waiting for it), covers them.
+            const long long first = !mma_cta ? issued : (issued > kStages ? issued - kStages : 0);
             for (long long i = first; i < issued; ++i) {
                 const uint32_t bar = full_bar(static_cast<int>(i % kStages));
                 const uint32_t par = static_cast<uint32_t>((i / kStages) & 1);
@@ -204,11 +268,11 @@ bf16_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant
         __syncwarp();
     } else if (warp == 1) {
         // ============================================================ MMA issuer
-        if (ptx::elect_one()) {
+        if (mma_cta && ptx::elect_one()) {
             int stage = 0, buf = 0;
             uint32_t phase = 0, tphase = 0;
             bool ok = true;
-            const uint32_t idesc = bf16_idesc(kTileX, kBN);
+            const uint32_t idesc = bf16_idesc(kTileX * kCtaGroup, kBN);
             for (int t = t_first; ok && t < num_tiles; t += t_step) {
                 Tile tl;
                 if (!TM::decode(t, p, prefix, tl)) continue;
@@ -220,17 +284,27 @@ bf16_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant
                     const uint32_t sx = s_base + stage * L::kStageBytes;
                     const uint64_t dx = sw128_desc(sx);
                     const uint64_t dy = sw128_desc(sx + L::kXBytes);
+                    if constexpr (kPair) {
 #pragma unroll
-                    for (int k = 0; k < kBf16BlockK / 16; ++k)
-                        ptx::mma_f16(dtm, dx + 2u * k, dy + 2u * k, idesc, (kb > kb_begin || k > 0) ? 1u : 0u);
-                    ptx::mma_commit(empty_bar(stage));
+                        for (int k = 0; k < kBf16BlockK / 16; ++k)
+                            ptx::mma_f16_pair(dtm, dx + 2u * k, dy + 2u * k, idesc, (kb > kb_begin || k > 0) ? 1u : 0u);
+                        ptx::mma_commit_pair(empty_bar(stage), 0x3);
+                    } else {
+#pragma unroll
+                        for (int k = 0; k < kBf16BlockK / 16; ++k)
+                            ptx::mma_f16(dtm, dx + 2u * k, dy + 2u * k, idesc, (kb > kb_begin || k > 0) ? 1u : 0u);
+                        ptx::mma_commit(empty_bar(stage));
+                    }
                     if (++stage == kStages) { stage = 0; phase ^= 1u; }
                 }
                 if (!ok) break;
-                ptx::mma_commit(tfull_bar(buf));
+                if constexpr (kPair) ptx::mma_commit_pair(tfull_bar(buf), 0x3);
+                else ptx::mma_commit(tfull_bar(buf));
                 if (++buf == kAccBufs) { buf = 0; tphase ^= 1u; }
             }
-            ptx::mma_commit(mma_done_bar);
+            // the commit is issued even when nothing ran, so every wait on it is uniform
+            if constexpr (kPair) ptx::mma_commit_pair(mma_done_bar, 0x3);
+            else ptx::mma_commit(mma_done_bar);
         }
         __syncwarp();
     } else if (warp >= kEpiWarp0) {
@@ -265,8 +339,8 @@ bf16_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant
                 have_split_tile = true;
                 break;   // one tile per cluster
             }
-            const int my_tok = tl.tok0 + lrow;
-            const bool row_ok = my_tok < tl.tok_end;
+            const int my_tok = tl.tok0 + my_row0 + lrow;
+            const bool row_ok = my_tok < tl.tok_end && ((tl.store >> pair_rank) & 1);
             const size_t row_base = kLayout == kMasked ? static_cast<size_t>(tl.g) * p.M : 0;
             __nv_bfloat16 *drow = p.d + (row_base + my_tok) * static_cast<size_t>(p.N);
 #pragma unroll 1
@@ -293,10 +367,14 @@ bf16_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant
                     }
                 }
             }
-            // the accumulator is free for the MMA warp's next tile
+            // the accumulator is free for the MMA warp's next tile (released on the
+            // MMA CTA's barrier: remote for a pair's second CTA)
             ptx::tc_fence_before();
             __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(tempty_bar(buf));
+            if (lane == 0) {
+                if (kPair && !mma_cta) ptx::mbar_arrive_remote(leader_addr(tempty_bar(buf)));
+                else ptx::mbar_arrive(tempty_bar(buf));
+            }
             if (++buf == kAccBufs) { buf = 0; tphase ^= 1u; }
         }
         if (clustered) {
@@ -394,9 +472,11 @@ bf16_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant
     __syncwarp();
     ptx::tc_fence_before();
     __syncthreads();
+    if constexpr (kPair) ptx::cluster_sync_all();   // no CTA leaves while its peer may touch its smem
     if (warp == 1) {
         ptx::tc_fence_after();
-        ptx::tmem_dealloc(tmem_base, L::kTmemCols);
+        if constexpr (kPair) ptx::tmem_dealloc_pair(tmem_base, L::kTmemCols);
+        else ptx::tmem_dealloc(tmem_base, L::kTmemCols);
     }
 }
 

@@ -273,7 +273,10 @@ struct TileMap {
                 wb = local / width;
                 const int g0 = block_group(p, 2 * pair), g1 = block_group(p, 2 * pair + 1);
                 g = g0 >= 0 ? g0 : g1;
-                if (g < 0) return false;
+                if (g < 0) {                 // both blocks are padding: no work
+                    tl.tok0 = pair * kTokRows;   // callers may still inspect the pair's first row
+                    return false;
+                }
                 store = (g0 == g ? 1 : 0) | (g1 == g ? 2 : 0);
             } else {
                 const int q = (t - first) / nw;

@@ -105,6 +105,45 @@ def test_contiguous_matches_oracle(counts, N, K):
     compare(d, _ref(prob), valid)
 
 
+def _bf16_child(kind, args, pairs):
+    """Runs one BF16 problem in a child process with DG_BF16_PAIRS forcing CTA
+    pairs (1) or single-CTA tiles (0); returns the launch log."""
+    import os, subprocess, sys
+    make = {"dense": "W.make_bf16_dense(*%r, seed=21)",
+            "contiguous": "W.make_bf16_contiguous(*%r[:3], seed=22, gaps=%r[3])"}[kind]
+    code = ("import sys; sys.path[:0] = [%r, %r]\n"
+            "import numpy as np, test_gpu_bf16 as T, workloads as W\n"
+            "from gpu_util import compare\n"
+            "import oracle; oracle.build()\n"
+            "p = " + make + "\n"
+            "d = T._run(p).double().cpu().numpy()\n"
+            "valid = np.ones(p.d_shape(), bool) if p.layout == 'dense' else "
+            "np.broadcast_to((p.m_indices >= 0)[:, None], p.d_shape())\n"
+            "compare(d, T._ref(p), valid)\n"
+            "import moe_grouped_gemm_fp32_b200 as dg; assert dg.dg_get_device_status(clear=True) == 0\n"
+            "print('OK')\n") % ((os.path.dirname(os.path.dirname(__file__)), os.path.dirname(__file__))
+                                  + ((args,) if kind == "dense" else (args, args)))
+    env = dict(os.environ, DG_BF16_PAIRS="1" if pairs else "0", DG_VERBOSE="1")
+    r = subprocess.run([sys.executable, "-c", code], env=env, capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0 and "OK" in r.stdout, r.stdout + r.stderr
+    return r.stderr
+
+
+@pytest.mark.parametrize("kind,args", [("dense", (512, 448, 512)), ("dense", (300, 520, 136)),
+                                       ("dense", (1024, 7168, 256)),
+                                       ("contiguous", ([130, 200, 5, 300, 129], 448, 384, None)),
+                                       ("contiguous", ([200, 100, 300], 256, 256, [2, 0, 0])),
+                                       ("contiguous", ([5, 130], 384, 128, [3, 1]))])
+@pytest.mark.parametrize("pairs", [True, False])
+def test_cta_pairs_and_single_tiles(kind, args, pairs):
+    """Both tile kinds of the dense and contiguous BF16 layouts, each forced in
+    a child process: 256-row CTA-pair tiles (second passes where a pair's two
+    blocks belong to different groups; pairs of padding blocks with no work)
+    and 128-row single-CTA tiles."""
+    log = _bf16_child(kind, args, pairs)
+    assert ("ctas/mma=2" if pairs else "ctas/mma=1") in log
+
+
 @pytest.mark.parametrize("masked_m,Mmax,N,K", [([0, 1, 64, 200, 130], 200, 384, 512),
                                                ([256] * 3, 256, 4096, 256), ([5, 0], 8, 136, 64)])
 def test_masked_matches_oracle_and_leaves_rows(masked_m, Mmax, N, K):

@@ -57,6 +57,28 @@ def test_dense_small_m_split_k(M, K):
     _run_full(W.make_dense(M, 2112, K, seed=7 + M, outliers=True))
 
 
+def test_split_k_needs_four_k_blocks_per_cta():
+    """The split-K factor of swap-mode tiles leaves every CTA at least four
+    K-blocks: K = 512 (4 K-blocks) runs unsplit, K = 1024 splits at most in two,
+    K = 7168 splits; each result matches the oracle (child process, DG_VERBOSE
+    reports the launch)."""
+    import os, re, subprocess, sys
+    code = ("import sys; sys.path[:0] = [%r, %r]\n"
+            "import workloads as W, oracle\n"
+            "from gpu_util import DeviceProblem, compare, to_f64, valid_mask\n"
+            "for i, (M, N, K) in enumerate([(128, 256, 512), (64, 2112, 1024), (64, 2112, 7168)]):\n"
+            "    p = W.make_dense(M, N, K, seed=40 + i, outliers=True)\n"
+            "    d = to_f64(DeviceProblem(p).run())\n"
+            "    compare(d, oracle.solve(p), valid_mask(p))\n"
+            "    print('OK', K, flush=True)\n"
+            % (os.path.dirname(os.path.dirname(__file__)), os.path.dirname(__file__)))
+    r = subprocess.run([sys.executable, "-c", code], env=dict(os.environ, DG_VERBOSE="1"),
+                       capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0 and r.stdout.count("OK") == 3, r.stdout + r.stderr
+    split = {int(k): int(s) for k, s in re.findall(r"K=(\d+) G=1 .*? split=(\d+)", r.stderr)}
+    assert split[512] == 1 and split[1024] <= 2 and split[7168] >= 2, split
+
+
 @pytest.mark.parametrize("M,N", [(512, 256), (384, 384), (1024, 1152)])
 def test_dense_normal_mode(M, N):
     _run_full(W.make_dense(M, N, 1024, seed=M + N))
@@ -110,12 +132,18 @@ def test_contiguous(counts, N, K):
     _run_full(W.make_contiguous(counts, N, K, seed=sum(counts) + N))
 
 
-@pytest.mark.parametrize("counts,N,K", [([130, 200, 5, 300, 129], 448, 384), ([128, 256], 2112, 512)])
-def test_contiguous_cta_pairs(counts, N, K):
+@pytest.mark.parametrize("counts,N,K,gaps", [([130, 200, 5, 300, 129], 448, 384, None),
+                                             ([128, 256], 2112, 512, None),
+                                             # blocks 2 and 3 are both padding: a pair tile with
+                                             # no work; blocks 4|5 hold groups 1|2 (second pass)
+                                             ([200, 100, 300], 256, 256, [2, 0, 0]),
+                                             ([5, 130], 384, 256, [3, 1])])
+def test_contiguous_cta_pairs(counts, N, K, gaps):
     """The CTA-pair contiguous path (the default for N > 128 and K >= 4096),
     forced on at small K in a child process: second passes for pair tiles
-    whose two 128-row blocks belong to different groups."""
-    _run_contiguous_child(counts, N, K, pairs=True)
+    whose two 128-row blocks belong to different groups, and pair tiles whose
+    two blocks are both padding (whole unused blocks of the caller's buffer)."""
+    _run_contiguous_child(counts, N, K, pairs=True, gaps=gaps)
 
 
 @pytest.mark.parametrize("counts,N,K", [([130, 200, 5, 300, 129], 384, 4096), ([1] * 7, 256, 4096)])
@@ -124,15 +152,15 @@ def test_contiguous_single_cta_tiles(counts, N, K):
     _run_contiguous_child(counts, N, K, pairs=False)
 
 
-def _run_contiguous_child(counts, N, K, pairs):
+def _run_contiguous_child(counts, N, K, pairs, gaps=None):
     import os, subprocess, sys
     code = ("import sys; sys.path[:0] = [%r, %r]\n"
             "import workloads as W, oracle\n"
             "from gpu_util import DeviceProblem, compare, to_f64, valid_mask\n"
-            "p = W.make_contiguous(%r, %d, %d, seed=77)\n"
+            "p = W.make_contiguous(%r, %d, %d, seed=77, gaps=%r)\n"
             "dp = DeviceProblem(p); dp.fill_sentinel(); d = to_f64(dp.run())\n"
             "compare(d, oracle.solve(p), valid_mask(p)); print('OK')\n"
-            % (os.path.dirname(os.path.dirname(__file__)), os.path.dirname(__file__), counts, N, K))
+            % (os.path.dirname(os.path.dirname(__file__)), os.path.dirname(__file__), counts, N, K, gaps))
     env = dict(os.environ, DG_CONTIG_PAIRS="1" if pairs else "0", DG_VERBOSE="1")
     r = subprocess.run([sys.executable, "-c", code], env=env, capture_output=True, text=True, timeout=300)
     assert r.returncode == 0 and "OK" in r.stdout, r.stdout + r.stderr

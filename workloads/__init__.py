@@ -177,15 +177,18 @@ def make_dense(M: int, N: int, K: int, seed: int, outliers: bool = False,
 
 
 def make_contiguous(counts, N: int, K: int, seed: int, name: str = "",
-                    poison: bool = True) -> Problem:
+                    poison: bool = True, gaps=None) -> Problem:
     """M-grouped contiguous problem with explicit per-group token counts.
 
     Group g's rows are packed back to back and padded to a multiple of 128;
-    padding rows carry m_indices = -1, NaN bytes in A and NaN scales."""
+    padding rows carry m_indices = -1, NaN bytes in A and NaN scales.
+    ``gaps[g]`` whole 128-row blocks of padding follow group g's rows (a
+    caller's fixed-size buffer with unused blocks)."""
     rng = np.random.default_rng(seed)
     counts = [int(c) for c in counts]
     G = len(counts)
-    padded = [(c + ALIGN_M - 1) // ALIGN_M * ALIGN_M for c in counts]
+    gaps = [0] * G if gaps is None else [int(x) for x in gaps]
+    padded = [(c + ALIGN_M - 1) // ALIGN_M * ALIGN_M + ALIGN_M * x for c, x in zip(counts, gaps)]
     M_total = int(sum(padded))
     a32 = _normal(rng, (sum(counts), K))
     b32 = _normal(rng, (G * N, K))
@@ -473,13 +476,15 @@ def make_bf16_dense(M: int, N: int, K: int, seed: int, name: str = "") -> BF16Pr
     return BF16Problem("dense", M, N, K, 1, a, b[None], name=name)
 
 
-def make_bf16_contiguous(counts, N: int, K: int, seed: int, name: str = "") -> BF16Problem:
+def make_bf16_contiguous(counts, N: int, K: int, seed: int, name: str = "", gaps=None) -> BF16Problem:
     """Contiguous layout: groups packed back to back, each padded to 128 rows;
-    padding rows hold BF16 NaN and m_indices -1."""
+    padding rows hold BF16 NaN and m_indices -1.  ``gaps[g]`` whole 128-row
+    blocks of padding follow group g's rows."""
     rng = np.random.default_rng(seed)
     counts = [int(c) for c in counts]
     G = len(counts)
-    padded = [(c + ALIGN_M - 1) // ALIGN_M * ALIGN_M for c in counts]
+    gaps = [0] * G if gaps is None else [int(x) for x in gaps]
+    padded = [(c + ALIGN_M - 1) // ALIGN_M * ALIGN_M + ALIGN_M * x for c, x in zip(counts, gaps)]
     M_total = int(sum(padded))
     a_all = _bf16_bits(_normal(rng, (sum(counts), K)))
     b = _bf16_bits(_normal(rng, (G * N, K))).reshape(G, N, K)
