@@ -224,7 +224,10 @@ bf16_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant
             for (int t = t_first; ok && t < num_tiles; t += t_step) {
                 Tile tl;
                 if (!TM::decode(t, p, prefix, tl)) {
-                    if (kLayout == kContiguous && __ldg(p.m_indices + tl.tok0) >= p.G)
+                    // a block whose group index is out of range (single-CTA tiles;
+                    // on CTA pairs, where a tile without work leaves tl unset, the
+                    // set-up pass over every block records it)
+                    if (kLayout == kContiguous && !TM::kPairedGroups && __ldg(p.m_indices + tl.tok0) >= p.G)
                         record_status(p.status, kStatusInvalid, kSiteBadGroup);
                     continue;
                 }

@@ -273,10 +273,7 @@ struct TileMap {
                 wb = local / width;
                 const int g0 = block_group(p, 2 * pair), g1 = block_group(p, 2 * pair + 1);
                 g = g0 >= 0 ? g0 : g1;
-                if (g < 0) {                 // both blocks are padding: no work
-                    tl.tok0 = pair * kTokRows;   // callers may still inspect the pair's first row
-                    return false;
-                }
+                if (g < 0) return false;
                 store = (g0 == g ? 1 : 0) | (g1 == g ? 2 : 0);
             } else {
                 const int q = (t - first) / nw;
@@ -626,7 +623,10 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant_
             for (int t = t_first; ok && t < num_tiles; t += t_step) {
                 Tile tl;
                 if (!TM::decode(t, p, prefix, tl)) {
-                    if (kLayout == kContiguous && __ldg(p.m_indices + tl.tok0) >= p.G)
+                    // a block whose group index is out of range (single-CTA tiles;
+                    // on CTA pairs, where a tile without work leaves tl unset, the
+                    // set-up pass over every block records it)
+                    if (kLayout == kContiguous && !TM::kPairedGroups && __ldg(p.m_indices + tl.tok0) >= p.G)
                         record_status(p.status, kStatusInvalid, kSiteBadGroup);
                     continue;
                 }
