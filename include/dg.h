@@ -248,7 +248,9 @@ DG_API dg_status_t dg_bf16_gemm_nt(const void *a, const void *b, void *d, int M,
 /* Contiguous M-grouped BF16: a [M_total, K] (groups packed, each padded to 128
  * rows), b [G, N, K], d [M_total, N], m_indices [M_total] int32 on the device
  * with the same precondition and padding rules as the FP8 contiguous call.
- * M_total % 128 == 0. */
+ * Here the 256-row block pairs (and their limit of 1024 pairs holding two
+ * different groups) apply to every call with N > 128, at least two blocks and
+ * G < 1024, whatever K.  M_total % 128 == 0. */
 DG_API dg_status_t dg_m_grouped_bf16_gemm_nt_contiguous(const void *a, const void *b, void *d,
                                                         const int32_t *m_indices, int M_total,
                                                         int N, int K, int G, void *stream);
