@@ -180,6 +180,18 @@ def test_contiguous_equals_per_group_dense(oracle_lib):
     assert np.isfinite(d[~pad]).all()              # NaN padding never leaks
 
 
+def test_contiguous_with_whole_padding_blocks(oracle_lib):
+    """Whole padding blocks between groups change nothing for the groups' rows:
+    the same groups without the gaps give the same outputs, and padding rows
+    stay unwritten."""
+    gapped = W.make_contiguous([200, 100, 300], N=136, K=256, seed=6, gaps=[2, 0, 1])
+    plain = W.make_contiguous([200, 100, 300], N=136, K=256, seed=6)
+    d, e = oracle_lib.solve(gapped), oracle_lib.solve(plain)
+    for g in range(3):
+        assert np.array_equal(d[gapped.m_indices == g], e[plain.m_indices == g])
+    assert np.isnan(d[gapped.m_indices < 0]).all()
+
+
 def test_masked_equals_per_group_dense(oracle_lib):
     prob = W.make_masked([0, 7, 64, 65], Mmax=64 + 16, N=160, K=256, seed=4)
     d = oracle_lib.solve(prob)

@@ -52,6 +52,25 @@ def test_contiguous_structure():
         assert len(ids) <= 1
 
 
+def test_contiguous_gap_blocks():
+    """gaps[g] whole 128-row padding blocks follow group g (a caller's buffer
+    with unused blocks); without gaps the generator is unchanged."""
+    p = W.make_contiguous([200, 100, 300], N=64, K=128, seed=1, gaps=[2, 0, 1])
+    mi = p.m_indices
+    assert p.M == (256 + 256) + 128 + (384 + 128)
+    assert (mi[:200] == 0).all() and (mi[200:512] == -1).all()       # 56 rows + 2 whole blocks
+    assert (mi[512:612] == 1).all() and (mi[612:640] == -1).all()
+    assert (mi[640:940] == 2).all() and (mi[940:] == -1).all()
+    assert (p.a[mi < 0] == W.NAN_BYTE).all() and np.isnan(p.sfa[:, mi < 0]).all()
+    q, r = W.make_contiguous([200, 100, 300], N=64, K=128, seed=1), \
+        W.make_contiguous([200, 100, 300], N=64, K=128, seed=1, gaps=[0, 0, 0])
+    assert np.array_equal(q.a, r.a) and np.array_equal(q.m_indices, r.m_indices)
+    assert np.array_equal(q.b, p.b) and np.array_equal(p.a[mi == 2], q.a[q.m_indices == 2])
+    h = W.make_bf16_contiguous([5, 130], N=64, K=64, seed=3, gaps=[3, 1])
+    assert h.M == 128 * 4 + 256 + 128 and (h.m_indices[128:512] == -1).all()
+    assert (h.m_indices[512:642] == 1).all() and (h.m_indices[642:] == -1).all()
+
+
 def test_masked_structure():
     p = W.make_masked_uniform(16, 256, N=128, K=128, seed=5)
     assert p.masked_m.min() >= 0 and p.masked_m.max() <= 256
